@@ -1,0 +1,406 @@
+"""Benchmark of the Jano hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload large]
+                    [--impl reference] [--no-cpu-baseline] [--no-e2e]
+
+One step = one pass of the whole hot path over one batch of synthetic input
+(block scores over the latent history, level split of the per-token field,
+the 50-step schedule, KV-cache scatter of the Active tokens' fresh K/V and
+active-query attention over the whole cache), all through the C ABI.
+
+Metric: active-query attention TFLOP/s, FLOPs = 4 * N_act * N * d * heads,
+divided by the whole step's device time (max over ranks); the analyzer and
+scatter HBM GB/s and per-kernel times are reported beside it.  Every rank
+runs an independent replica of the workload (a different seed): the path
+has no data-path exchange, so N GPUs process N problems ("weak" scaling).
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead, on
+a bounded sample of the same workload, extrapolated stage by stage to the
+full workload.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "active-query attn TFLOP/s (% BF16 peak) at 75.6K tokens; analyzer HBM GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(w):
+    return {
+        "workload": f"{w.name}: latent {list(w.latent_shape)} fp32, blocks {list(w.block)}, "
+                    f"{w.n_tokens} tokens x {w.heads} heads x d={w.d} BF16, "
+                    f"levels {round(w.frac_active*100)}/{round((1-w.frac_active-w.frac_static)*100)}/"
+                    f"{round(w.frac_static*100)} from a smooth token field, Active-only step",
+        "tokens": w.n_tokens, "heads": w.heads, "d": w.d,
+        "latent": list(w.latent_shape), "block": list(w.block), "patch": list(w.patch),
+        "schedule": {"T": w.T, "warmup": w.warmup, "cooldown": w.cooldown,
+                     "period_moderate": w.period_moderate, "period_static": w.period_static},
+    }
+
+
+# ------------------------------------------------------------------ inputs
+def make_inputs(w, seed_shift=0):
+    import synth
+    import torch
+    TF, TH, TW = w.grid
+    lat = synth.latent_history(w.K, w.C, w.F, w.H, w.W, seed=w.seed + seed_shift)
+    field = synth.token_field(TF, TH, TW, seed=(w.seed + seed_shift) * 10 + 1, sigma=w.field_sigma)
+    N = w.n_tokens
+    n_cap = int(round(w.frac_active * 10000)) * N // 10000
+    base = (w.seed + seed_shift) * 1000
+    inp = dict(lat=torch.from_numpy(lat), field=torch.from_numpy(field),
+               q_act=synth.normal_bf16((n_cap, w.heads, w.d), base + 1),
+               k_act=synth.normal_bf16((n_cap, w.heads, w.d), base + 2),
+               v_act=synth.normal_bf16((n_cap, w.heads, w.d), base + 3))
+    k_cache = synth.normal_bf16((N, w.heads, w.d), base + 4)
+    v_cache = synth.normal_bf16((N, w.heads, w.d), base + 5)
+    return inp, k_cache, v_cache, n_cap
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r for r in csv.reader(io.StringIO(self.out or "")) if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows]
+        mx = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        busy = [v for v in sm if v > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows)}
+
+
+# ------------------------------------------------------------------ traffic record
+def traffic_for(kernel_src_rel):
+    """DRAM bytes per launch from the committed ncu record, if it was taken on
+    the current source of that kernel; else None."""
+    rec = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, kernel_src_rel)
+    if not (os.path.exists(rec) and os.path.exists(src)):
+        return None
+    with open(rec) as fh:
+        d = json.load(fh)
+    ent = d.get(kernel_src_rel)
+    if not ent:
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return ent.get("bytes_per_launch") if ent.get("source_sha") == sha else None
+
+
+# ------------------------------------------------------------------ CPU oracle
+def cpu_oracle_step_time(w, inp, k_cache, v_cache, budget_rows=8, rng_seed=0):
+    """Time the oracle stage by stage on a bounded sample, extrapolate each
+    stage to the full workload; returns (seconds per full step, sample text)."""
+    import oracle
+    import synth
+    oracle.build()
+    N, H, d = w.n_tokens, w.heads, w.d
+    lat = inp["lat"].numpy()
+    field = inp["field"].numpy()
+    est = 0.0
+    parts = []
+    # a1 on one frame-block slab of all snapshots/channels
+    bf = w.block[0]
+    slab = np.ascontiguousarray(lat[:, :, :bf])
+    t = time.perf_counter(); oracle.block_scores(slab, w.block); dt = time.perf_counter() - t
+    est += dt * (w.F / bf); parts.append(f"scores {bf}/{w.F} frames")
+    # a2 + a3 in full
+    t = time.perf_counter()
+    lv = oracle.classify(field, w.frac_active, w.frac_static)
+    pf, ph, pw = w.patch
+    off, idx, _ = oracle.build_schedule(lv, (w.F, w.H, w.W), w.patch, w.patch, w.T, w.warmup,
+                                        w.cooldown, w.period_moderate, w.period_static)
+    est += time.perf_counter() - t; parts.append("classify+schedule full")
+    n_act = int(off[w.warmup + 1] - off[w.warmup])
+    sel = idx[off[w.warmup]:off[w.warmup + 1]]
+    # a4 on 256 rows
+    m = min(256, n_act)
+    kb, vb = synth.bits_of(k_cache), synth.bits_of(v_cache)
+    ka, va = synth.bits_of(inp["k_act"][:m]), synth.bits_of(inp["v_act"][:m])
+    t = time.perf_counter(); oracle.kv_scatter(ka, va, sel[:m], kb, vb); dt = time.perf_counter() - t
+    est += dt * n_act / m; parts.append(f"scatter {m} rows")
+    # a5 on budget_rows rows x all heads x all keys
+    g = np.random.default_rng(rng_seed)
+    rows = np.sort(g.choice(n_act, size=min(budget_rows, n_act), replace=False)).astype(np.int32)
+    qb = synth.bits_of(inp["q_act"][:n_act])
+    t = time.perf_counter(); oracle.active_attention(qb, kb, vb, rows=rows); dt = time.perf_counter() - t
+    est += dt * n_act / rows.size; parts.append(f"attention {rows.size} rows x {H} heads x {N} keys")
+    flops = 4.0 * n_act * N * d * H
+    return est, flops, "; ".join(parts) + " (single-threaded fp64 C, extrapolated per stage)"
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return 0
+    inp, k_cache, v_cache, n_cap = make_inputs(w)
+    times = []
+    flops = None
+    sample = ""
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        est, flops, sample = cpu_oracle_step_time(w, inp, k_cache, v_cache,
+                                                  budget_rows=args.ref_rows, rng_seed=i)
+        if i >= args.warmup:
+            times.append(est)
+        log(f"reference step {i}: estimated full step {est:.1f} s (wall {time.perf_counter()-t0:.1f} s)")
+    t = statistics.mean(times)
+    value = flops / t / 1e12
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gpu(args, w, rank, world, local_rank, dist):
+    import torch
+    import kv_cache_analyzer_b200 as J
+    from kv_cache_analyzer_b200.pipeline import HotPath, KERNELS_PER_STEP
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(dev)
+    pk, pk_src = peaks()
+
+    inp, k_cache, v_cache, n_cap = make_inputs(w, seed_shift=rank)
+    hp = HotPath(K=w.K, C=w.C, latent_geom=J.Geometry(w.F, w.H, w.W, w.block, w.patch),
+                 token_geom=J.Geometry(w.F, w.H, w.W, w.patch, w.patch), heads=w.heads, d=w.d,
+                 frac_active=w.frac_active, frac_static=w.frac_static,
+                 sched=J.Schedule(w.T, w.warmup, w.cooldown, w.period_moderate, w.period_static),
+                 device=dev, stream=stream)
+    hp.set_activations(n_cap)
+    with torch.cuda.stream(stream):
+        hp.lat.copy_(inp["lat"])
+        hp.field.copy_(inp["field"])
+        hp.q_act.copy_(inp["q_act"]); hp.k_act.copy_(inp["k_act"]); hp.v_act.copy_(inp["v_act"])
+        hp.k_cache.copy_(k_cache); hp.v_cache.copy_(v_cache)
+    stream.synchronize()
+    hp.plan()
+    step = w.warmup                       # first interleaved step: Active tokens only
+    _, n_act = hp.due(step)
+    assert n_act <= n_cap, (n_act, n_cap)
+    flops = 4.0 * n_act * w.n_tokens * w.d * w.heads
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    # ---- warm-up
+    for _ in range(args.warmup):
+        hp.run_step_kernels(step)
+    stream.synchronize()
+    code = J.device_error(stream)
+    if code:
+        raise RuntimeError(f"device error after warm-up: {J.jano_status_str(code)}")
+
+    # ---- timed: device-resident inputs, per-stage events on the launching stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            hp.run_step_kernels(step, evs[i])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    total_ms = start.elapsed_time(end)
+    stage = np.array([[e[k].elapsed_time(e[k + 1]) for k in range(5)] for e in evs])  # ms
+    # stage columns: scores, classify, schedule, scatter, attention
+    stage_ms = stage.mean(axis=0)
+    t_max = total_ms
+    if dist is not None:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt.item())
+    ms_per_step = t_max / args.steps
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    code = J.device_error(stream)
+    if code:
+        raise RuntimeError(f"device error in timed region: {J.jano_status_str(code)}")
+
+    # ---- end to end: host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        host = {k: v.pin_memory() for k, v in inp.items()}
+        host["q_act"] = host["q_act"][:n_act]; host["k_act"] = host["k_act"][:n_act]
+        host["v_act"] = host["v_act"][:n_act]
+        host_out = torch.empty(hp.out.shape, dtype=hp.out.dtype).pin_memory()
+        for _ in range(max(1, args.warmup)):
+            hp.step_from_host(step, host, host_out)
+        stream.synchronize()
+        barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(args.steps):
+            hp.step_from_host(step, host, host_out)
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_ms = s2.elapsed_time(e2)
+        if dist is not None:
+            tt = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        e2e = {"value": world * flops / (e2e_ms / args.steps * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": HotPath.h2d_bytes(host),
+               "d2h_bytes_per_step": host_out.numel() * host_out.element_size()}
+
+    if rank != 0:
+        return 0
+
+    # ---- per-kernel figures and roofline of the dominant kernel (attention)
+    hbm = pk["hbm_gbs"]
+    bf16_sus = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    lat_bytes = float(np.prod(w.latent_shape)) * 4
+    scat_bytes = 4.0 * n_act * w.heads * w.d * 2
+    att_tflops = flops / (stage_ms[4] * 1e-3) / 1e12
+    kernels = {
+        "block_scores": {"ms": stage_ms[0], "GB/s": lat_bytes / (stage_ms[0] * 1e-3) / 1e9,
+                         "algorithmic_bytes": lat_bytes},
+        "classify": {"ms": stage_ms[1], "n": w.n_tokens},
+        "build_schedule": {"ms": stage_ms[2], "T": w.T},
+        "kv_scatter": {"ms": stage_ms[3], "GB/s": scat_bytes / (stage_ms[3] * 1e-3) / 1e9,
+                       "algorithmic_bytes": scat_bytes},
+        "active_attention": {"ms": stage_ms[4], "TFLOP/s": att_tflops, "flops": flops,
+                             "n_active": n_act},
+    }
+    for k in ("block_scores", "kv_scatter"):
+        kernels[k]["frac_of_hbm"] = kernels[k]["GB/s"] / hbm
+    kernels["active_attention"]["frac_of_burst_peak"] = att_tflops / pk["bf16_tflops"]
+    roofline = {"bound": "tensor", "achieved": att_tflops, "peak": bf16_sus, "unit": "TFLOP/s",
+                "frac": att_tflops / bf16_sus,
+                "traffic": traffic_for("kv_cache_analyzer_b200/csrc/attention.cu"),
+                "peak_kind": f"{pk_src} sustained cuBLAS bf16 (kernel timed inside a long step)",
+                "kernel": "active_attention"}
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        t0 = time.perf_counter()
+        est, fl, sample = cpu_oracle_step_time(w, inp, k_cache, v_cache, budget_rows=args.ref_rows)
+        cpu = {"value": fl / est / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+               "sample": sample, "wall_s": time.perf_counter() - t0}
+
+    cfg = workload_config(w)
+    cfg.update({"n_active": n_act, "global_batch": world, "parallelism": f"replicas x{world}",
+                "l2": "no flush: the per-step working set (K/V cache 1.5 GB, Q/K/V act 0.6 GB) "
+                      "is far larger than the 126 MB L2"})
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": cfg, "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": e2e, "gpu_launches": KERNELS_PER_STEP * args.steps, "clocks": clk.summary(),
+            "kernels": kernels, "peaks": {"source": pk_src, "hbm_gbs": hbm,
+                                          "bf16_tflops": pk["bf16_tflops"],
+                                          "bf16_tflops_sustained": bf16_sus}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="large")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=8)
+    args = ap.parse_args()
+
+    import synth
+    w = synth.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        log(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE")
+
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                 device_id=torch.device("cuda", local_rank))
+        dist = tdist
+    try:
+        return run_gpu(args, w, rank, world, local_rank, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,213 @@
+/*
+ * jano.h -- C ABI of libjano, the B200 (sm_100a) library for the
+ * data-parallel hot path of Jano ("Jano: Adaptive Diffusion Generation with
+ * Early-stage Convergence Awareness", arXiv 2603.00519, as summarised on the
+ * gist.science pages in nl/fr/pt/zh/ko).
+ *
+ * The hot path has two parts:
+ *   1. the block-wise complexity analyzer and its three-level split
+ *      (jano_block_scores, jano_classify) plus the interleaved token schedule
+ *      built from it (jano_build_schedule);
+ *   2. the per-step partial-token attention: fresh K/V of the due tokens are
+ *      scattered into a persistent full-sequence cache (jano_kv_scatter) and
+ *      only the due (active) queries attend over the whole cache
+ *      (jano_active_attention), their outputs going back to their token rows.
+ *
+ * Conventions shared by every entry point
+ *   - All pointers named *device* below are device pointers on the current
+ *     CUDA device; `stream` is a cudaStream_t passed as void* (NULL = the
+ *     legacy default stream).  Every launch is asynchronous on `stream`.
+ *   - The caller owns every buffer.  The library allocates no device or host
+ *     memory; scratch space, where an entry point needs some, is passed in by
+ *     the caller and sized by a *_workspace_bytes query.
+ *   - Argument errors are detected on the host before anything is launched
+ *     and returned synchronously; nothing is written in that case.  A failed
+ *     launch returns JANO_ECUDA.  Errors that only the device can see (an
+ *     index out of range, a non-finite score, an invalid level) set a sticky
+ *     per-device error word that jano_get_device_error() reads and clears.
+ *     Kernels never trap: an offending element is skipped, and every wait
+ *     inside a kernel is bounded in time.
+ *   - Layouts are dense and row-major, the last index fastest.
+ *   - Token order: a token is a pf x ph x pw patch of the latent, and token
+ *     id t = (ft*TH + th)*TW + tw with TF=F/pf, TH=H/ph, TW=W/pw.  Q/K/V/O
+ *     rows are [tokens][heads][d] BF16, one contiguous row of heads*d values
+ *     per token; the KV cache is kept in token order.
+ */
+#ifndef JANO_H
+#define JANO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define JANO_API __attribute__((visibility("default")))
+#else
+#define JANO_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    JANO_OK = 0,
+    JANO_EINVAL = 1,        /* bad argument value or NULL pointer            */
+    JANO_ESHAPE = 2,        /* inconsistent sizes (e.g. F not divisible by pf) */
+    JANO_EALIGN = 3,        /* pointer not 16-byte aligned                    */
+    JANO_EUNSUPPORTED = 4,  /* valid but not implemented (e.g. d not 64/128)  */
+    JANO_ENONFINITE = 5,    /* device: a score was NaN or infinite            */
+    JANO_EINDEX = 6,        /* device: an index or level was out of range     */
+    JANO_ETIMEOUT = 7,      /* device: a bounded internal wait gave up (a bug) */
+    JANO_ECUDA = 8          /* a CUDA runtime call or launch failed           */
+} jano_status;
+
+/* Latent geometry: latent dims (F frames, H rows, W columns), analyzer block
+ * dims (bf, bh, bw) and token patch dims (pf, ph, pw), all in latent
+ * elements.  Blocks at the far edges may be partial; F, H, W must be
+ * multiples of pf, ph, pw. */
+typedef struct {
+    int F, H, W;
+    int bf, bh, bw;
+    int pf, ph, pw;
+} jano_geom;
+
+/* Interleaved schedule: T sampling steps; the first `warmup` and the last
+ * `cooldown` are full steps; in between, Moderate tokens refresh every
+ * `period_moderate` steps and Static tokens every `period_static` steps. */
+typedef struct {
+    int T, warmup, cooldown, period_moderate, period_static;
+} jano_sched_cfg;
+
+/* ------------------------------------------------------------------------
+ * jano_block_scores -- block-wise complexity score.
+ * Pages: zh technical summary 2.1 (3D frame x height x width blocks;
+ * temporal and spatial gradients; second-order differences over the first K
+ * steps, about 10% of sampling, combined into a per-block score); nl
+ * technical summary, Methodologie 1 "Implementatie"; pt 2.A.
+ *
+ *   S_b = mean over k=1..K-1 and every (c,f,h,w) in block b of
+ *         |x_{k+1} - 2 x_k + x_{k-1}| + w_temporal |D_f x_k|
+ *                                     + w_spatial sqrt(D_h x_k^2 + D_w x_k^2)
+ *
+ * D_* are forward differences, 0 where the neighbour is outside the tensor
+ * (it may lie in the next block); edge blocks average over their real
+ * elements.  The usual weights are 0.5 and 0.5.
+ *
+ * lat     device fp32 [K+1][C][F][H][W], 16-byte aligned; W % 4 == 0.
+ * K       index of the last snapshot (K+1 snapshots); K >= 2.
+ * scores  device fp32 [nBf*nBh*nBw], nBx = ceil(X/bx), block id
+ *         (bf_i*nBh + bh_i)*nBw + bw_i.  Deterministic (fixed reduction
+ *         order, no atomics).
+ * Patch dims in `g` are not used here.
+ * ---------------------------------------------------------------------- */
+JANO_API jano_status jano_block_scores(const float *lat, int K, int C, const jano_geom *g,
+                              float w_temporal, float w_spatial, float *scores,
+                              void *stream);
+
+/* ------------------------------------------------------------------------
+ * jano_classify -- three convergence levels (Level 1 Static, 2 Moderate,
+ * 3 Active).  Pages: nl technical summary, Methodologie 1 "Resultaat";
+ * zh 2.2 item 1; ko 2.B.
+ *
+ * Blocks are ordered by the key (score ascending, block index ascending;
+ * -0 ranks as +0).  With bp_X = round(frac_X * 10000) and
+ * n_X = floor(bp_X * n_blocks / 10000), the first n_S blocks are Static,
+ * the last n_A Active, the rest Moderate.  frac_active + frac_static <= 1.
+ *
+ * scores  device fp32 [n_blocks] (any finite values).
+ * levels  device uint8 [n_blocks], written with 1, 2 or 3.
+ * A NaN or infinite score raises JANO_ENONFINITE on the device error word
+ * and leaves `levels` unspecified.  One thread block; no scratch memory.
+ * ---------------------------------------------------------------------- */
+JANO_API jano_status jano_classify(const float *scores, int n_blocks, float frac_active,
+                          float frac_static, uint8_t *levels, void *stream);
+
+/* ------------------------------------------------------------------------
+ * jano_build_schedule -- block levels -> token levels -> per-step lists of
+ * due tokens for all T steps (CSR).  Pages: nl technical summary,
+ * Methodologie 2 (warm-up; Level 1 rarely, Level 2 intermittently, Level 3
+ * every step; cool-down); zh 2.2 item 2; fr 2.B "Pipeline Intercalé".
+ *
+ * A token takes the level of the block holding its first latent element.
+ * Step s is full when s < warmup or s >= T - cooldown; otherwise, with
+ * j = s - warmup, Level 3 is due, Level 2 when (j+1) % period_moderate == 0
+ * and Level 1 when (j+1) % period_static == 0.
+ *
+ * block_levels  device uint8 [n_blocks] (values 1..3; others raise EINDEX
+ *               on the device error word and count as Static).
+ * offsets       device int32 [T+1]: step s lists idx[offsets[s]..offsets[s+1]).
+ * idx           device int32, capacity idx_capacity >= T * n_tokens; the due
+ *               token ids of each step in ascending order.
+ * token_levels  device uint8 [n_tokens] or NULL.
+ * workspace     device scratch of jano_build_schedule_workspace_bytes(g)
+ *               bytes, 16-byte aligned; its contents need not be initialised
+ *               and are meaningless afterwards.
+ * ---------------------------------------------------------------------- */
+JANO_API size_t jano_build_schedule_workspace_bytes(const jano_geom *g);
+JANO_API jano_status jano_build_schedule(const uint8_t *block_levels, const jano_geom *g,
+                                const jano_sched_cfg *c, int32_t *offsets,
+                                int32_t *idx, size_t idx_capacity,
+                                uint8_t *token_levels, void *workspace,
+                                size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * jano_kv_scatter -- write the fresh K/V rows of the due tokens into the
+ * persistent full-sequence cache: k_cache[idx[i]] = k_act[i],
+ * v_cache[idx[i]] = v_act[i], bit for bit, both in one pass.
+ * Pages: nl technical summary, Methodologie 2 "KV Cache Mechanisme" (the
+ * K/V of frozen tokens are kept and reused); zh 2.2 item 3; pt 2.B.
+ *
+ * k_act, v_act      device BF16 [n_act][heads][d].
+ * idx               device int32 [n_act], distinct ids in [0, n_tokens)
+ *                   (jano_build_schedule emits ascending ones).  An id out of
+ *                   range raises JANO_EINDEX on the device error word and
+ *                   its row is skipped.  Duplicate ids: unspecified winner.
+ * k_cache, v_cache  device BF16 [n_tokens][heads][d]; must not overlap the
+ *                   act buffers.  All four 16-byte aligned; heads*d % 8 == 0.
+ * n_act == 0 is a no-op.
+ * ---------------------------------------------------------------------- */
+JANO_API jano_status jano_kv_scatter(const void *k_act, const void *v_act, const int32_t *idx,
+                            int n_act, int heads, int d, void *k_cache,
+                            void *v_cache, int n_tokens, void *stream);
+
+/* ------------------------------------------------------------------------
+ * jano_active_attention -- attention of only the active queries over the
+ * whole cached K/V, outputs written back to their token rows:
+ *   out[idx[i], h, :] = softmax_j(scale * q_act[i,h,:] . k_cache[j,h,:])
+ *                       @ v_cache[:, h, :]        over all n_tokens j.
+ * Pages: nl technical summary, Methodologie 2 "KV Cache Mechanisme" (cached
+ * K/V concatenated with the active queries; no position restoration since
+ * attention does not depend on the order of keys/values); ko 2.B; pt 2.B.
+ * The cache is kept in token order, so no concatenation copy is made.
+ *
+ * q_act             device BF16 [n_act][heads][d] (the due tokens' queries,
+ *                   in the order of idx).
+ * k_cache, v_cache  device BF16 [n_tokens][heads][d].
+ * idx               device int32 [n_act]: output row of each query; out of
+ *                   range raises JANO_EINDEX and the row is skipped.
+ * out               device BF16 [n_tokens][heads][d]; only rows idx[] are
+ *                   written.  May not alias the inputs.
+ * d in {64, 128}; BF16 in, fp32 accumulate and softmax, BF16 out;
+ * no mask, no bias; scale is normally 1/sqrt(d).  All pointers 16-byte
+ * aligned.  n_act == 0 is a no-op.
+ * ---------------------------------------------------------------------- */
+JANO_API jano_status jano_active_attention(const void *q_act, const void *k_cache,
+                                  const void *v_cache, const int32_t *idx,
+                                  int n_act, int n_tokens, int heads, int d,
+                                  float scale, void *out, void *stream);
+
+/* Synchronises `stream`, returns the first device-side error recorded on the
+ * current device since the last call (JANO_OK if none) and clears it. */
+JANO_API jano_status jano_get_device_error(void *stream);
+
+/* Static English text for a status code. */
+JANO_API const char *jano_status_str(jano_status s);
+
+/* Library version, major*10000 + minor*100 + patch. */
+JANO_API int jano_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JANO_H */

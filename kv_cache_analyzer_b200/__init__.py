@@ -1,0 +1,251 @@
+"""kv_cache_analyzer_b200 -- Python binding of libjano, the B200 (sm_100a)
+library for the data-parallel hot path of Jano (block-wise complexity
+analyzer, three-level token schedule, KV-cache scatter and active-query
+attention).
+
+The functions named ``jano_*`` mirror the C ABI in ``include/jano.h`` one to
+one: they only marshal torch tensors (device memory) and the current CUDA
+stream into the C call and turn a non-OK status into ``JanoError``.  The
+lower-case helpers below them allocate outputs with torch and call those.
+Every step of the path runs in the library's CUDA kernels; there is no CPU
+or PyTorch fallback, and importing a function fails loudly when the library
+is not built.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+
+import torch
+
+__all__ = [
+    "JanoError", "jano_geom", "jano_sched_cfg", "lib", "library_path",
+    "jano_block_scores", "jano_classify", "jano_build_schedule_workspace_bytes",
+    "jano_build_schedule", "jano_kv_scatter", "jano_active_attention",
+    "jano_get_device_error", "jano_status_str", "jano_version",
+    "Geometry", "Schedule", "block_scores", "classify", "build_schedule",
+    "kv_scatter", "active_attention", "device_error",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libjano.so")
+
+STATUS_NAMES = {0: "JANO_OK", 1: "JANO_EINVAL", 2: "JANO_ESHAPE", 3: "JANO_EALIGN",
+                4: "JANO_EUNSUPPORTED", 5: "JANO_ENONFINITE", 6: "JANO_EINDEX",
+                7: "JANO_ETIMEOUT", 8: "JANO_ECUDA"}
+EXPORTS = ("jano_block_scores", "jano_classify", "jano_build_schedule_workspace_bytes",
+           "jano_build_schedule", "jano_kv_scatter", "jano_active_attention",
+           "jano_get_device_error", "jano_status_str", "jano_version")
+
+
+class JanoError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+class jano_geom(C.Structure):
+    _fields_ = [(n, C.c_int) for n in ("F", "H", "W", "bf", "bh", "bw", "pf", "ph", "pw")]
+
+
+class jano_sched_cfg(C.Structure):
+    _fields_ = [(n, C.c_int) for n in ("T", "warmup", "cooldown", "period_moderate", "period_static")]
+
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """Load libjano.so (built in-tree by ``python -m kv_cache_analyzer_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise RuntimeError(f"libjano.so is not built at {library_path}; "
+                               "run `python -m kv_cache_analyzer_b200.build`")
+        L = C.CDLL(library_path)
+        P, i, f, z = C.c_void_p, C.c_int, C.c_float, C.c_size_t
+        G, S = C.POINTER(jano_geom), C.POINTER(jano_sched_cfg)
+        L.jano_block_scores.argtypes = [P, i, i, G, f, f, P, P]
+        L.jano_classify.argtypes = [P, i, f, f, P, P]
+        L.jano_build_schedule_workspace_bytes.argtypes = [G]
+        L.jano_build_schedule_workspace_bytes.restype = z
+        L.jano_build_schedule.argtypes = [P, G, S, P, P, z, P, P, z, P]
+        L.jano_kv_scatter.argtypes = [P, P, P, i, i, i, P, P, i, P]
+        L.jano_active_attention.argtypes = [P, P, P, P, i, i, i, i, f, P, P]
+        L.jano_get_device_error.argtypes = [P]
+        L.jano_status_str.argtypes = [i]
+        L.jano_status_str.restype = C.c_char_p
+        L.jano_version.argtypes = []
+        for fn in ("jano_block_scores", "jano_classify", "jano_build_schedule",
+                   "jano_kv_scatter", "jano_active_attention", "jano_get_device_error",
+                   "jano_version"):
+            getattr(L, fn).restype = C.c_int
+        _lib = L
+    return _lib
+
+
+def _stream(stream) -> C.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dev(t: torch.Tensor | None, name: str, dtype=None) -> C.c_void_p | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return C.c_void_p(t.data_ptr())
+
+
+def _check(fn: str, code: int) -> None:
+    if code != 0:
+        raise JanoError(fn, code)
+
+
+# ---------------------------------------------------------------- C ABI mirror
+def jano_block_scores(lat, K, C_, geom, w_temporal, w_spatial, scores, stream=None):
+    _check("jano_block_scores", lib().jano_block_scores(
+        _dev(lat, "lat", torch.float32), K, C_, C.byref(geom), w_temporal, w_spatial,
+        _dev(scores, "scores", torch.float32), _stream(stream)))
+
+
+def jano_classify(scores, n_blocks, frac_active, frac_static, levels, stream=None):
+    _check("jano_classify", lib().jano_classify(
+        _dev(scores, "scores", torch.float32), n_blocks, frac_active, frac_static,
+        _dev(levels, "levels", torch.uint8), _stream(stream)))
+
+
+def jano_build_schedule_workspace_bytes(geom) -> int:
+    return int(lib().jano_build_schedule_workspace_bytes(C.byref(geom)))
+
+
+def jano_build_schedule(block_levels, geom, cfg, offsets, idx, idx_capacity, token_levels,
+                        workspace, ws_bytes, stream=None):
+    _check("jano_build_schedule", lib().jano_build_schedule(
+        _dev(block_levels, "block_levels", torch.uint8), C.byref(geom), C.byref(cfg),
+        _dev(offsets, "offsets", torch.int32), _dev(idx, "idx", torch.int32), idx_capacity,
+        _dev(token_levels, "token_levels", torch.uint8), _dev(workspace, "workspace"),
+        ws_bytes, _stream(stream)))
+
+
+def jano_kv_scatter(k_act, v_act, idx, n_act, heads, d, k_cache, v_cache, n_tokens, stream=None):
+    _check("jano_kv_scatter", lib().jano_kv_scatter(
+        _dev(k_act, "k_act", torch.bfloat16), _dev(v_act, "v_act", torch.bfloat16),
+        _dev(idx, "idx", torch.int32), n_act, heads, d,
+        _dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
+        n_tokens, _stream(stream)))
+
+
+def jano_active_attention(q_act, k_cache, v_cache, idx, n_act, n_tokens, heads, d, scale, out,
+                          stream=None):
+    _check("jano_active_attention", lib().jano_active_attention(
+        _dev(q_act, "q_act", torch.bfloat16), _dev(k_cache, "k_cache", torch.bfloat16),
+        _dev(v_cache, "v_cache", torch.bfloat16), _dev(idx, "idx", torch.int32), n_act,
+        n_tokens, heads, d, scale, _dev(out, "out", torch.bfloat16), _stream(stream)))
+
+
+def jano_get_device_error(stream=None) -> int:
+    return int(lib().jano_get_device_error(_stream(stream)))
+
+
+def jano_status_str(code: int) -> str:
+    return lib().jano_status_str(code).decode()
+
+
+def jano_version() -> int:
+    return int(lib().jano_version())
+
+
+# ---------------------------------------------------------------- helpers
+@dataclass(frozen=True)
+class Geometry:
+    """Latent dims, analyzer block and token patch (latent elements)."""
+    F: int
+    H: int
+    W: int
+    block: tuple = (1, 4, 4)
+    patch: tuple = (1, 2, 2)
+
+    def c(self) -> jano_geom:
+        return jano_geom(self.F, self.H, self.W, *self.block, *self.patch)
+
+    @property
+    def n_blocks(self) -> int:
+        bf, bh, bw = self.block
+        return (-(-self.F // bf)) * (-(-self.H // bh)) * (-(-self.W // bw))
+
+    @property
+    def n_tokens(self) -> int:
+        pf, ph, pw = self.patch
+        return (self.F // pf) * (self.H // ph) * (self.W // pw)
+
+
+@dataclass(frozen=True)
+class Schedule:
+    T: int = 50
+    warmup: int = 5
+    cooldown: int = 5
+    period_moderate: int = 2
+    period_static: int = 4
+
+    def c(self) -> jano_sched_cfg:
+        return jano_sched_cfg(self.T, self.warmup, self.cooldown, self.period_moderate,
+                              self.period_static)
+
+
+def block_scores(lat: torch.Tensor, geom: Geometry, w_temporal=0.5, w_spatial=0.5,
+                 out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    K1, Cc = lat.shape[0], lat.shape[1]
+    if out is None:
+        out = torch.empty(geom.n_blocks, dtype=torch.float32, device=lat.device)
+    jano_block_scores(lat, K1 - 1, Cc, geom.c(), w_temporal, w_spatial, out, stream)
+    return out
+
+
+def classify(scores: torch.Tensor, frac_active: float, frac_static: float,
+             out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty(scores.numel(), dtype=torch.uint8, device=scores.device)
+    jano_classify(scores, scores.numel(), frac_active, frac_static, out, stream)
+    return out
+
+
+def build_schedule(block_levels: torch.Tensor, geom: Geometry, sched: Schedule,
+                   stream=None, workspace: torch.Tensor | None = None):
+    """-> (offsets int32 [T+1], idx int32 [T*N capacity], token_levels uint8 [N])."""
+    dev = block_levels.device
+    g = geom.c()
+    N = geom.n_tokens
+    ws_bytes = jano_build_schedule_workspace_bytes(g)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    offsets = torch.empty(sched.T + 1, dtype=torch.int32, device=dev)
+    idx = torch.empty(sched.T * N, dtype=torch.int32, device=dev)
+    tl = torch.empty(N, dtype=torch.uint8, device=dev)
+    jano_build_schedule(block_levels, g, sched.c(), offsets, idx, idx.numel(), tl, workspace,
+                        workspace.numel(), stream)
+    return offsets, idx, tl
+
+
+def kv_scatter(k_act, v_act, idx, k_cache, v_cache, stream=None) -> None:
+    n_act = idx.numel()
+    N, H, d = k_cache.shape
+    jano_kv_scatter(k_act, v_act, idx, n_act, H, d, k_cache, v_cache, N, stream)
+
+
+def active_attention(q_act, k_cache, v_cache, idx, out, scale=None, stream=None) -> None:
+    n_act = idx.numel()
+    N, H, d = k_cache.shape
+    if scale is None:
+        scale = d ** -0.5
+    jano_active_attention(q_act, k_cache, v_cache, idx, n_act, N, H, d, scale, out, stream)
+
+
+def device_error(stream=None) -> int:
+    return jano_get_device_error(stream)

@@ -1,0 +1,183 @@
+// jano_api.cu -- the exported C ABI of libjano: argument validation on the
+// host, then one or more asynchronous launches on the caller's stream.  See
+// include/jano.h for the contract of each entry point.
+#include <cmath>
+#include <cstdint>
+#include <climits>
+
+#include "jano_common.cuh"
+
+namespace jano {
+
+__device__ int g_device_error = JANO_OK;
+
+int* device_error_word() {
+    static int* addr[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<int*>(p);
+    }
+    return addr[dev];
+}
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+jano_status from_cuda(cudaError_t e) { return e == cudaSuccess ? JANO_OK : JANO_ECUDA; }
+
+jano_status check_geom(const jano_geom* g, bool need_patch) {
+    if (!g) return JANO_EINVAL;
+    if (g->F < 1 || g->H < 1 || g->W < 1 || g->bf < 1 || g->bh < 1 || g->bw < 1)
+        return JANO_EINVAL;
+    if (need_patch) {
+        if (g->pf < 1 || g->ph < 1 || g->pw < 1) return JANO_EINVAL;
+        if (g->F % g->pf || g->H % g->ph || g->W % g->pw) return JANO_ESHAPE;
+        const long long nt = (long long)(g->F / g->pf) * (g->H / g->ph) * (g->W / g->pw);
+        if (nt > INT_MAX) return JANO_EUNSUPPORTED;
+    }
+    const long long nb = (long long)((g->F + g->bf - 1) / g->bf) * ((g->H + g->bh - 1) / g->bh) *
+                         ((g->W + g->bw - 1) / g->bw);
+    if (nb > INT_MAX) return JANO_EUNSUPPORTED;
+    return JANO_OK;
+}
+
+}  // namespace
+}  // namespace jano
+
+using namespace jano;
+
+extern "C" {
+
+jano_status jano_block_scores(const float* lat, int K, int C, const jano_geom* g,
+                              float w_temporal, float w_spatial, float* scores,
+                              void* stream) {
+    if (!lat || !scores) return JANO_EINVAL;
+    if (K < 2 || C < 1) return JANO_EINVAL;
+    if (!std::isfinite(w_temporal) || !std::isfinite(w_spatial)) return JANO_EINVAL;
+    const jano_status gs = check_geom(g, false);
+    if (gs != JANO_OK) return gs;
+    if (g->W % 4) return JANO_EUNSUPPORTED;
+    if (!aligned16(lat)) return JANO_EALIGN;
+    if (!analyzer_supported(*g)) return JANO_EUNSUPPORTED;
+    if ((long long)g->F > 65535 || (long long)((g->H + g->bh - 1) / g->bh) > 65535)
+        return JANO_EUNSUPPORTED;
+    int* err = device_error_word();
+    if (!err) return JANO_ECUDA;
+    return from_cuda(launch_block_scores(lat, K, C, *g, w_temporal, w_spatial, scores, err,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+jano_status jano_classify(const float* scores, int n_blocks, float frac_active,
+                          float frac_static, uint8_t* levels, void* stream) {
+    if (!scores || !levels || n_blocks < 1) return JANO_EINVAL;
+    if (!(frac_active >= 0.0f && frac_active <= 1.0f) || !(frac_static >= 0.0f && frac_static <= 1.0f))
+        return JANO_EINVAL;
+    const long long bpA = std::llround((double)frac_active * 10000.0);
+    const long long bpS = std::llround((double)frac_static * 10000.0);
+    if (bpA + bpS > 10000) return JANO_EINVAL;
+    const long long nA = bpA * n_blocks / 10000;
+    const long long nS = bpS * n_blocks / 10000;
+    int* err = device_error_word();
+    if (!err) return JANO_ECUDA;
+    return from_cuda(launch_classify(scores, n_blocks, nS, (long long)n_blocks - nA, levels, err,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+size_t jano_build_schedule_workspace_bytes(const jano_geom* g) {
+    if (check_geom(g, true) != JANO_OK) return 0;
+    return schedule_workspace_bytes(*g);
+}
+
+jano_status jano_build_schedule(const uint8_t* block_levels, const jano_geom* g,
+                                const jano_sched_cfg* c, int32_t* offsets, int32_t* idx,
+                                size_t idx_capacity, uint8_t* token_levels, void* workspace,
+                                size_t ws_bytes, void* stream) {
+    if (!block_levels || !c || !offsets || !idx || !workspace) return JANO_EINVAL;
+    const jano_status gs = check_geom(g, true);
+    if (gs != JANO_OK) return gs;
+    if (c->T < 1 || c->warmup < 0 || c->cooldown < 0 || c->warmup + c->cooldown > c->T ||
+        c->period_moderate < 1 || c->period_static < 1)
+        return JANO_EINVAL;
+    if (c->T > 65535) return JANO_EUNSUPPORTED;
+    const long long nt = (long long)(g->F / g->pf) * (g->H / g->ph) * (g->W / g->pw);
+    if (nt * c->T > INT_MAX) return JANO_EUNSUPPORTED;
+    if (idx_capacity < (size_t)(nt * c->T)) return JANO_EINVAL;
+    if (ws_bytes < schedule_workspace_bytes(*g)) return JANO_EINVAL;
+    if (!aligned16(workspace)) return JANO_EALIGN;
+    int* err = device_error_word();
+    if (!err) return JANO_ECUDA;
+    return from_cuda(launch_build_schedule(block_levels, *g, *c, offsets, idx, token_levels,
+                                           workspace, err, static_cast<cudaStream_t>(stream)));
+}
+
+jano_status jano_kv_scatter(const void* k_act, const void* v_act, const int32_t* idx, int n_act,
+                            int heads, int d, void* k_cache, void* v_cache, int n_tokens,
+                            void* stream) {
+    if (n_act < 0 || heads < 1 || d < 1 || n_tokens < 1) return JANO_EINVAL;
+    if (n_act == 0) return JANO_OK;
+    if (!k_act || !v_act || !idx || !k_cache || !v_cache) return JANO_EINVAL;
+    const long long row_bytes = (long long)heads * d * 2;
+    if (row_bytes % 16) return JANO_EUNSUPPORTED;
+    if (row_bytes > INT_MAX) return JANO_EUNSUPPORTED;
+    if (!aligned16(k_act) || !aligned16(v_act) || !aligned16(k_cache) || !aligned16(v_cache))
+        return JANO_EALIGN;
+    int* err = device_error_word();
+    if (!err) return JANO_ECUDA;
+    return from_cuda(launch_kv_scatter(k_act, v_act, idx, n_act, (int)row_bytes, k_cache, v_cache,
+                                       n_tokens, err, static_cast<cudaStream_t>(stream)));
+}
+
+jano_status jano_active_attention(const void* q_act, const void* k_cache, const void* v_cache,
+                                  const int32_t* idx, int n_act, int n_tokens, int heads, int d,
+                                  float scale, void* out, void* stream) {
+    if (n_act < 0 || n_tokens < 1 || heads < 1) return JANO_EINVAL;
+    if (!(scale > 0.0f) || !std::isfinite(scale)) return JANO_EINVAL;
+    if (d != 64 && d != 128) return JANO_EUNSUPPORTED;
+    if (heads > 65535) return JANO_EUNSUPPORTED;
+    if (n_act == 0) return JANO_OK;
+    if (!q_act || !k_cache || !v_cache || !idx || !out) return JANO_EINVAL;
+    if (!aligned16(q_act) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return JANO_EALIGN;
+    int* err = device_error_word();
+    if (!err) return JANO_ECUDA;
+    return from_cuda(launch_active_attention(q_act, k_cache, v_cache, idx, n_act, n_tokens, heads,
+                                             d, scale, out, err, static_cast<cudaStream_t>(stream)));
+}
+
+jano_status jano_get_device_error(void* stream) {
+    int* err = device_error_word();
+    if (!err) return JANO_ECUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return JANO_ECUDA;
+    int v = JANO_OK;
+    if (cudaMemcpy(&v, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return JANO_ECUDA;
+    if (v != JANO_OK) {
+        const int zero = JANO_OK;
+        if (cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+            return JANO_ECUDA;
+    }
+    return static_cast<jano_status>(v);
+}
+
+const char* jano_status_str(jano_status s) {
+    switch (s) {
+        case JANO_OK: return "ok";
+        case JANO_EINVAL: return "invalid argument";
+        case JANO_ESHAPE: return "inconsistent shape";
+        case JANO_EALIGN: return "pointer not 16-byte aligned";
+        case JANO_EUNSUPPORTED: return "unsupported configuration";
+        case JANO_ENONFINITE: return "non-finite score";
+        case JANO_EINDEX: return "index or level out of range";
+        case JANO_ETIMEOUT: return "device wait timed out";
+        case JANO_ECUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+int jano_version(void) { return 100; }
+
+}  // extern "C"

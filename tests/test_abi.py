@@ -1,0 +1,93 @@
+"""The C-ABI library loads and exports every symbol include/jano.h declares,
+and host-side argument validation rejects bad calls without touching a GPU."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "jano.h")).read()
+    return re.findall(r"JANO_API\s+[\w\s\*]+?\b(jano_\w+)\s*\(", txt)
+
+
+@pytest.fixture(scope="module")
+def jl():
+    from kv_cache_analyzer_b200 import build
+    build.build()
+    import kv_cache_analyzer_b200 as j
+    return j
+
+
+def test_header_declares_the_boundary():
+    names = set(_declared())
+    for fn in ("jano_block_scores", "jano_classify", "jano_build_schedule",
+               "jano_kv_scatter", "jano_active_attention"):
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol(jl):
+    L = jl.lib()
+    for name in _declared():
+        assert hasattr(L, name), name
+    assert set(_declared()) == set(jl.EXPORTS)
+
+
+def test_status_strings_and_version(jl):
+    assert jl.jano_version() >= 100
+    assert jl.jano_status_str(0) == "ok"
+    assert "index" in jl.jano_status_str(6)
+
+
+def test_workspace_query_is_host_only(jl):
+    g = jl.Geometry(21, 90, 160, (1, 4, 4), (1, 2, 2))
+    n = jl.jano_build_schedule_workspace_bytes(g.c())
+    # token levels (75600 B) + two int32 [3][74] tables, 16-byte rounded
+    assert n == 75600 + 2 * 896
+    bad = jl.Geometry(21, 91, 160, (1, 4, 4), (1, 2, 2))     # H not divisible by ph
+    assert jl.jano_build_schedule_workspace_bytes(bad.c()) == 0
+
+
+def test_host_validation_rejects_before_any_launch(jl):
+    L = jl.lib()
+    nil = C.c_void_p(0)
+    fake = C.c_void_p(256)          # never dereferenced: validation fails first
+    # d not in {64, 128}
+    assert L.jano_active_attention(fake, fake, fake, fake, 10, 100, 2, 96, 0.1, fake, nil) == 4
+    # non-positive scale
+    assert L.jano_active_attention(fake, fake, fake, fake, 10, 100, 2, 128, 0.0, fake, nil) == 1
+    # misaligned pointer
+    assert L.jano_active_attention(C.c_void_p(258), fake, fake, fake, 10, 100, 2, 128, 0.1, fake, nil) == 3
+    # n_act == 0 is a no-op that succeeds without a device
+    assert L.jano_active_attention(nil, nil, nil, nil, 0, 100, 2, 128, 0.1, nil, nil) == 0
+    assert L.jano_kv_scatter(nil, nil, nil, 0, 2, 128, nil, nil, 100, nil) == 0
+    assert L.jano_kv_scatter(fake, fake, fake, -1, 2, 128, fake, fake, 100, nil) == 1
+    # row of heads*d BF16 not a multiple of 16 bytes
+    assert L.jano_kv_scatter(fake, fake, fake, 3, 1, 4, fake, fake, 100, nil) == 4
+    # classify fractions out of range / summing above 1
+    assert L.jano_classify(fake, 10, 0.7, 0.7, fake, nil) == 1
+    assert L.jano_classify(fake, 10, -0.1, 0.2, fake, nil) == 1
+    assert L.jano_classify(fake, 0, 0.1, 0.2, fake, nil) == 1
+    # block scores: K < 2, W not a multiple of 4
+    g = jl.Geometry(4, 32, 32).c()
+    assert L.jano_block_scores(fake, 1, 16, C.byref(g), 0.5, 0.5, fake, nil) == 1
+    g2 = jl.Geometry(4, 32, 30, (1, 4, 4), (1, 2, 2)).c()
+    assert L.jano_block_scores(fake, 5, 16, C.byref(g2), 0.5, 0.5, fake, nil) == 4
+    # schedule: warm-up + cool-down longer than T, index capacity too small
+    g3 = jl.Geometry(4, 32, 32).c()
+    bad = jl.Schedule(T=4, warmup=3, cooldown=2).c()
+    assert L.jano_build_schedule(fake, C.byref(g3), C.byref(bad), fake, fake, 10**6, nil, fake,
+                                 10**6, nil) == 1
+    ok = jl.Schedule(T=4, warmup=1, cooldown=1).c()
+    assert L.jano_build_schedule(fake, C.byref(g3), C.byref(ok), fake, fake, 10, nil, fake,
+                                 10**6, nil) == 1
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch, jl):
+    monkeypatch.setattr(jl, "library_path", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(jl, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        jl.lib()
