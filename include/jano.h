@@ -151,6 +151,36 @@ JANO_API jano_status jano_build_schedule(const uint8_t *block_levels, const jano
                                 size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
+ * jano_build_schedule_noalloc -- jano_build_schedule for callers that cannot
+ * allocate device memory.  The Jano pages have no counterpart: this is a
+ * deployment convenience, not part of the method.
+ *
+ * Some callers cannot call cudaMalloc or any allocating routine where they
+ * build the schedule (code running inside someone else's CUDA-graph
+ * capture, runtimes without a device allocator, hosts whose memory pool
+ * forbids side allocations).  This variant takes the same inputs and outputs
+ * as jano_build_schedule but no workspace: its scratch is a file-scope
+ * __device__ array of 1 MiB inside the library, which every GPU that loads
+ * the library holds until the process exits.  It allocates nothing.
+ *
+ * Limit: the scratch the geometry needs (jano_build_schedule_workspace_bytes)
+ * must not exceed 1 MiB, i.e. about 1.04 million tokens; larger geometries
+ * return JANO_EUNSUPPORTED and launch nothing.  Other errors are those of
+ * jano_build_schedule.
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.
+ * Sharing: every call on a device uses the same array and it keeps the last
+ * call's contents (the builder needs no zeroed scratch).  Calls whose
+ * launches overlap on the GPU (different streams, no ordering between them)
+ * race on the array; order them on one stream or with events.
+ * ---------------------------------------------------------------------- */
+JANO_API jano_status jano_build_schedule_noalloc(const uint8_t *block_levels, const jano_geom *g,
+                                         const jano_sched_cfg *c, int32_t *offsets,
+                                         int32_t *idx, size_t idx_capacity,
+                                         uint8_t *token_levels, void *stream);
+
+/* ------------------------------------------------------------------------
  * jano_kv_scatter -- write the fresh K/V rows of the due tokens into the
  * persistent full-sequence cache: k_cache[idx[i]] = k_act[i],
  * v_cache[idx[i]] = v_act[i], bit for bit, both in one pass.

@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "JanoError", "jano_geom", "jano_sched_cfg", "lib", "library_path",
     "jano_block_scores", "jano_classify", "jano_build_schedule_workspace_bytes",
-    "jano_build_schedule", "jano_kv_scatter", "jano_active_attention",
+    "jano_build_schedule", "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention",
     "jano_get_device_error", "jano_status_str", "jano_version",
     "Geometry", "Schedule", "block_scores", "classify", "build_schedule",
     "kv_scatter", "active_attention", "device_error",
@@ -35,7 +35,7 @@ STATUS_NAMES = {0: "JANO_OK", 1: "JANO_EINVAL", 2: "JANO_ESHAPE", 3: "JANO_EALIG
                 4: "JANO_EUNSUPPORTED", 5: "JANO_ENONFINITE", 6: "JANO_EINDEX",
                 7: "JANO_ETIMEOUT", 8: "JANO_ECUDA"}
 EXPORTS = ("jano_block_scores", "jano_classify", "jano_build_schedule_workspace_bytes",
-           "jano_build_schedule", "jano_kv_scatter", "jano_active_attention",
+           "jano_build_schedule", "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention",
            "jano_get_device_error", "jano_status_str", "jano_version")
 
 
@@ -71,6 +71,7 @@ def lib() -> C.CDLL:
         L.jano_build_schedule_workspace_bytes.argtypes = [G]
         L.jano_build_schedule_workspace_bytes.restype = z
         L.jano_build_schedule.argtypes = [P, G, S, P, P, z, P, P, z, P]
+        L.jano_build_schedule_noalloc.argtypes = [P, G, S, P, P, z, P, P]
         L.jano_kv_scatter.argtypes = [P, P, P, i, i, i, P, P, i, P]
         L.jano_active_attention.argtypes = [P, P, P, P, i, i, i, i, f, P, P]
         L.jano_get_device_error.argtypes = [P]
@@ -78,7 +79,7 @@ def lib() -> C.CDLL:
         L.jano_status_str.restype = C.c_char_p
         L.jano_version.argtypes = []
         for fn in ("jano_block_scores", "jano_classify", "jano_build_schedule",
-                   "jano_kv_scatter", "jano_active_attention", "jano_get_device_error",
+                   "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention", "jano_get_device_error",
                    "jano_version"):
             getattr(L, fn).restype = C.c_int
         _lib = L
@@ -132,6 +133,19 @@ def jano_build_schedule(block_levels, geom, cfg, offsets, idx, idx_capacity, tok
         _dev(offsets, "offsets", torch.int32), _dev(idx, "idx", torch.int32), idx_capacity,
         _dev(token_levels, "token_levels", torch.uint8), _dev(workspace, "workspace"),
         ws_bytes, _stream(stream)))
+
+
+def jano_build_schedule_noalloc(block_levels, geom, cfg, offsets, idx, idx_capacity, token_levels,
+                                stream=None):
+    """jano_build_schedule without a workspace argument: for callers that
+    cannot allocate device memory.  The library's own 1 MiB device array
+    serves as scratch (geometries up to about 1.04 million tokens); calls
+    overlapping on the GPU race on it, and the first call on a device should
+    come before any stream capture."""
+    _check("jano_build_schedule_noalloc", lib().jano_build_schedule_noalloc(
+        _dev(block_levels, "block_levels", torch.uint8), C.byref(geom), C.byref(cfg),
+        _dev(offsets, "offsets", torch.int32), _dev(idx, "idx", torch.int32), idx_capacity,
+        _dev(token_levels, "token_levels", torch.uint8), _stream(stream)))
 
 
 def jano_kv_scatter(k_act, v_act, idx, n_act, heads, d, k_cache, v_cache, n_tokens, stream=None):
