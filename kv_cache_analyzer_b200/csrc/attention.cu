@@ -7,22 +7,29 @@
 //   out[idx[i], h] = softmax_j(scale * q_act[i,h] . k_cache[j,h]) @ v_cache[:, h]
 //
 // Flash-style forward on the 5th-generation tensor cores.  One CTA per
-// (128-query tile, head); 6 warps:
-//   warp 0     TMA producer: Q tile once, then K_j / V_j tiles (128 keys x d)
-//              into a 2-stage shared-memory ring (128-byte swizzle, boxes of
-//              64 columns), completion counted on mbarriers.
-//   warp 1     allocates 512 TMEM columns; one lane issues every tcgen05.mma:
-//              S_j = Q K_j^T (both K-major in smem) into TMEM buffer j%2, then
-//              O += P_{j-1} V_{j-1} with P read from TMEM (A operand) and V
-//              MN-major from smem.  tcgen05.commit arrives on the barriers
-//              that free smem stages and hand S to the softmax warps.
-//   warps 2-5  softmax: thread = one query row = one TMEM lane.  Reads its S
-//              row (128 fp32) with tcgen05.ld, masks the ragged last key tile,
-//              keeps the running max in the log2 domain and rescales O in TMEM
-//              only when the max grows by more than 2^8 (lazy rescale), writes
-//              P as packed BF16 into TMEM, and finally normalises O and stores
-//              the BF16 row to out[idx[i]].
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,256+d) P0, P1 (64 each).
+// (pair of 128-query tiles, head); 12 warps:
+//   warps 0-3, 4-7  softmax warpgroups WG0 / WG1, one per query tile:
+//              thread = one query row = one TMEM lane.  Per key tile the row's
+//              S (128 fp32) is read from TMEM in two halves, the running max
+//              is kept in the log2 domain and O is rescaled in TMEM only when
+//              the max grows by more than 2^8 (lazy rescale), P is written as
+//              packed BF16 into the upper half of the row's S columns, and at
+//              the end O is normalised and stored as BF16 to out[idx[i]].
+//   warp 8     TMA producer: both Q tiles once, then K_j, V_j (128 keys x d)
+//              into a 4-slot shared-memory ring (128-byte swizzle, boxes of
+//              64 columns); completion counted on mbarriers.
+//   warp 9     allocates 512 TMEM columns; one lane issues every tcgen05.mma
+//              in the ping-pong order
+//                 S0_0 S1_0 | PV0_{j-1} S0_j PV1_{j-1} S1_j | ... PV0 PV1
+//              so the tensor core runs one tile's MMAs while the other
+//              tile's softmax runs.  S = Q K^T reads Q and K K-major from
+//              smem; O += P V reads P from TMEM (A operand) and V MN-major
+//              from smem.  tcgen05.commit hands S to the softmax warps and
+//              frees ring slots.  Because S_i_j is issued after PV_i_{j-1},
+//              the softmax that sees S_i_j may rescale O_i safely.
+//   warps 10-11 idle.
+// TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [384,384+d);
+// P_i occupies columns [64,128) of S_i.
 // Every wait is bounded; on timeout the CTA records JANO_ETIMEOUT, drains its
 // own copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
@@ -36,10 +43,10 @@
 namespace jano {
 namespace {
 
-constexpr int BM = 128;            // queries per tile
+constexpr int BM = 128;            // queries per tile (two tiles per CTA)
 constexpr int BN = 128;            // keys per tile
-constexpr int kStages = 2;
-constexpr int kThreads = 192;
+constexpr int kSlots = 4;          // K/V ring slots
+constexpr int kThreads = 384;
 constexpr uint32_t kPanel = 128 * 128;   // bytes of one 128-row x 64-col BF16 panel
 constexpr long long kWaitLimit = 1ll << 31;  // cycles (~1 s)
 
@@ -47,30 +54,27 @@ template <int HD>
 struct Layout {
     static constexpr int kPanels = HD / 64;
     static constexpr uint32_t kTile = kPanels * kPanel;           // Q, K or V tile bytes
-    static constexpr uint32_t kQ = 0;
-    static constexpr uint32_t kK = kQ + kTile;
-    static constexpr uint32_t kV = kK + kStages * kTile;
-    static constexpr uint32_t kBar = kV + kStages * kTile;
+    static constexpr uint32_t kQ0 = 0;
+    static constexpr uint32_t kQ1 = kTile;
+    static constexpr uint32_t kRing = 2 * kTile;
+    static constexpr uint32_t kBar = kRing + kSlots * kTile;
     // barrier slots
     static constexpr int bQFull = 0;
-    static constexpr int bKFull = 1;
-    static constexpr int bKEmpty = bKFull + kStages;
-    static constexpr int bVFull = bKEmpty + kStages;
-    static constexpr int bVEmpty = bVFull + kStages;
-    static constexpr int bSFull = bVEmpty + kStages;   // [2]
-    static constexpr int bSFree = bSFull + 2;          // [2]
-    static constexpr int bPFull = bSFree + 2;          // [2]
-    static constexpr int bPVDone = bPFull + 2;         // [2]
-    static constexpr int bFinal = bPVDone + 2;
+    static constexpr int bFull = 1;                    // [kSlots]
+    static constexpr int bEmpty = bFull + kSlots;      // [kSlots]
+    static constexpr int bSFull = bEmpty + kSlots;     // [2]
+    static constexpr int bPFull = bSFull + 2;          // [2]
+    static constexpr int bOFull = bPFull + 2;          // [2]
+    static constexpr int bFinal = bOFull + 2;
     static constexpr int kNumBars = bFinal + 1;
     static constexpr uint32_t kMisc = kBar + 8 * kNumBars;        // tmem base, abort flag
     static constexpr uint32_t kBytes = kMisc + 16;
-    // 1 KB alignment slack; never below 116 KB so that at most one CTA sits on
-    // an SM and its 512 TMEM columns are never contended
-    static constexpr uint32_t kAlloc = (kBytes + 1024 > 116u * 1024) ? kBytes + 1024 : 116u * 1024;
+    static constexpr uint32_t kAlloc = kBytes + 1024;             // slack for 1 KB alignment
+    static_assert(kAlloc <= 227 * 1024, "shared memory budget");
     // TMEM columns
-    static constexpr uint32_t tS0 = 0, tS1 = 128, tO = 256;
-    static constexpr uint32_t tP0 = 256 + HD, tP1 = 256 + HD + 64;
+    __host__ __device__ static constexpr uint32_t tS(int i) { return i ? 128u : 0u; }
+    __host__ __device__ static constexpr uint32_t tO(int i) { return i ? 384u : 256u; }
+    static constexpr uint32_t tP = 64;                             // offset of P inside S
 };
 
 struct Ctl {
@@ -79,10 +83,10 @@ struct Ctl {
     int* err;
     __device__ uint32_t bar(int i) const { return bar0 + 8u * (uint32_t)i; }
     __device__ bool wait(int i, uint32_t parity) const {
-        if (mbar_try(i, parity)) return true;
+        if (ptx::mbar_try_wait(bar(i), parity)) return true;
         const long long t0 = clock64();
         for (;;) {
-            if (mbar_try(i, parity)) return true;
+            if (ptx::mbar_try_wait(bar(i), parity)) return true;
             if (*abort) return false;
             if (clock64() - t0 > kWaitLimit) {
                 *abort = 1;
@@ -91,7 +95,6 @@ struct Ctl {
             }
         }
     }
-    __device__ bool mbar_try(int i, uint32_t parity) const { return ptx::mbar_try_wait(bar(i), parity); }
     // Warp-uniform wait: lane 0 polls, the verdict is broadcast, so the
     // .sync.aligned tcgen05 operations that follow never run divergently.
     __device__ bool warp_wait(int i, uint32_t parity) const {
@@ -101,6 +104,92 @@ struct Ctl {
         return ok != 0;
     }
 };
+
+__device__ __forceinline__ float fmax4(float a, float b, float c, float d) {
+    return fmaxf(fmaxf(a, b), fmaxf(c, d));
+}
+
+// 64 consecutive TMEM columns of this warp's 32 lanes into registers.
+__device__ __forceinline__ void ld64(uint32_t taddr, uint32_t (&r)[64]) {
+    ptx::tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    ptx::tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+}
+
+// Row max of 64 values (8 independent chains); with kMask, keys >= valid
+// (the ragged last key tile) are left out.
+template <bool kMask>
+__device__ __forceinline__ float max64(const uint32_t (&s)[64], int valid) {
+    float m[8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a) m[a] = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 64; ++e)
+        if (!kMask || e < valid) m[e & 7] = fmaxf(m[e & 7], __uint_as_float(s[e]));
+    return fmaxf(fmax4(m[0], m[1], m[2], m[3]), fmax4(m[4], m[5], m[6], m[7]));
+}
+
+// p = 2^(s*c - m) for 64 values, packed to 32 BF16x2 words; returns sum(p).
+template <bool kMask>
+__device__ __forceinline__ float exp64(const uint32_t (&s)[64], int valid, float c, float m,
+                                       uint32_t* pk) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) {
+        float a = ptx::ex2(fmaf(__uint_as_float(s[e]), c, -m));
+        float b = ptx::ex2(fmaf(__uint_as_float(s[e + 1]), c, -m));
+        if (kMask && e >= valid) a = 0.f;
+        if (kMask && e + 1 >= valid) b = 0.f;
+        acc[(e >> 1) & 3] += a + b;
+        pk[e >> 1] = ptx::pack_bf16(a, b);
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// One key tile of one query row: row max over S (TMEM, two 64-column
+// halves), lazy O rescale, P = 2^(S*c - m) as BF16 into the upper half of
+// the row's S columns.  Warp-uniform control flow throughout.
+template <int HD, bool kMask>
+__device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, uint32_t tP, int j, int valid,
+                                             float c, float& m, float& l) {
+    uint32_t s[64];
+    ld64(tS, s);
+    ptx::tmem_wait_ld();
+    float mx = max64<kMask>(s, valid);
+    ld64(tS + 64, s);
+    ptx::tmem_wait_ld();
+    mx = fmaxf(mx, max64<kMask>(s, valid - 64));
+    const float mxs = mx * c;
+    // lazy rescale, decided per warp so the TMEM accesses stay warp-wide:
+    // lanes whose max did not grow past 2^8 keep their max (alpha = 1).
+    const bool want = mxs > m + 8.0f;
+    if (__any_sync(0xFFFFFFFFu, want)) {
+        const float m_new = want ? mxs : m;
+        if (j > 0) {
+            const float alpha = ptx::ex2(m - m_new);
+            l *= alpha;
+#pragma unroll
+            for (int q = 0; q < HD / 32; ++q) {
+                uint32_t o[32];
+                ptx::tmem_ld32(tO + 32 * q, o);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                ptx::tmem_st32(tO + 32 * q, o);
+            }
+            ptx::tmem_wait_st();
+        }
+        m = m_new;
+    }
+    // the upper half is still in registers: its P goes to P columns [32,64)
+    uint32_t pk[32];
+    l += exp64<kMask>(s, valid - 64, c, m, pk);
+    ptx::tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(pk));
+    ld64(tS, s);
+    ptx::tmem_wait_ld();
+    l += exp64<kMask>(s, valid, c, m, pk);
+    ptx::tmem_st32(tP, *reinterpret_cast<uint32_t(*)[32]>(pk));
+    ptx::tmem_wait_st();
+}
 
 template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -116,8 +205,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
     uint8_t* gbase = smem_raw + (base - raw);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt = blockIdx.x, head = blockIdx.y;
-    const int q0 = qt * BM;
+    const int head = blockIdx.y;
+    const int q0 = blockIdx.x * 2 * BM;                // first query row of tile 0
     const int nt = (n_tokens + BN - 1) / BN;
 
     Ctl ctl;
@@ -131,23 +220,20 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         ptx::prefetch_tmap(&tmK);
         ptx::prefetch_tmap(&tmV);
         ptx::mbar_init(ctl.bar(L::bQFull), 1);
-        for (int s = 0; s < kStages; ++s) {
-            ptx::mbar_init(ctl.bar(L::bKFull + s), 1);
-            ptx::mbar_init(ctl.bar(L::bKEmpty + s), 1);
-            ptx::mbar_init(ctl.bar(L::bVFull + s), 1);
-            ptx::mbar_init(ctl.bar(L::bVEmpty + s), 1);
+        for (int s = 0; s < kSlots; ++s) {
+            ptx::mbar_init(ctl.bar(L::bFull + s), 1);
+            ptx::mbar_init(ctl.bar(L::bEmpty + s), 1);
         }
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(ctl.bar(L::bSFull + s), 1);
-            ptx::mbar_init(ctl.bar(L::bSFree + s), 4);
             ptx::mbar_init(ctl.bar(L::bPFull + s), 4);
-            ptx::mbar_init(ctl.bar(L::bPVDone + s), 1);
+            ptx::mbar_init(ctl.bar(L::bOFull + s), 1);
         }
         ptx::mbar_init(ctl.bar(L::bFinal), 1);
         *ctl.abort = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == 9) {
         ptx::tmem_alloc(ptx::smem_u32(tmem_slot), 512);
         ptx::tmem_relinquish();
     }
@@ -156,88 +242,111 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
+    if (warp == 8) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            int lastK[kStages], lastV[kStages];
-            for (int s = 0; s < kStages; ++s) lastK[s] = lastV[s] = -1;
-            ptx::mbar_arrive_expect_tx(ctl.bar(L::bQFull), L::kTile);
-            for (int p = 0; p < L::kPanels; ++p)
-                ptx::tma_load_3d(base + L::kQ + p * kPanel, &tmQ, ctl.bar(L::bQFull), p * 64, head, q0);
-            for (int j = 0; j < nt; ++j) {
-                const int st = j % kStages;
-                const uint32_t ph = ((j / kStages) & 1) ^ 1;
-                if (!ctl.wait(L::bKEmpty + st, ph)) break;
-                ptx::mbar_arrive_expect_tx(ctl.bar(L::bKFull + st), L::kTile);
+            int last[kSlots];
+            for (int s = 0; s < kSlots; ++s) last[s] = -1;
+            ptx::mbar_arrive_expect_tx(ctl.bar(L::bQFull), 2 * L::kTile);
+            for (int p = 0; p < L::kPanels; ++p) {
+                ptx::tma_load_3d(base + L::kQ0 + p * kPanel, &tmQ, ctl.bar(L::bQFull), p * 64, head, q0);
+                ptx::tma_load_3d(base + L::kQ1 + p * kPanel, &tmQ, ctl.bar(L::bQFull), p * 64, head, q0 + BM);
+            }
+            // load sequence: K_0 V_0 K_1 V_1 ...; load n goes to slot n % kSlots
+            for (int n = 0; n < 2 * nt; ++n) {
+                const int s = n % kSlots;
+                if (!ctl.wait(L::bEmpty + s, ((n / kSlots) & 1) ^ 1)) break;
+                ptx::mbar_arrive_expect_tx(ctl.bar(L::bFull + s), L::kTile);
+                const CUtensorMap* tm = (n & 1) ? &tmV : &tmK;
                 for (int p = 0; p < L::kPanels; ++p)
-                    ptx::tma_load_3d(base + L::kK + st * L::kTile + p * kPanel, &tmK,
-                                     ctl.bar(L::bKFull + st), p * 64, head, j * BN);
-                lastK[st] = j;
-                if (!ctl.wait(L::bVEmpty + st, ph)) break;
-                ptx::mbar_arrive_expect_tx(ctl.bar(L::bVFull + st), L::kTile);
-                for (int p = 0; p < L::kPanels; ++p)
-                    ptx::tma_load_3d(base + L::kV + st * L::kTile + p * kPanel, &tmV,
-                                     ctl.bar(L::bVFull + st), p * 64, head, j * BN);
-                lastV[st] = j;
+                    ptx::tma_load_3d(base + L::kRing + s * L::kTile + p * kPanel, tm,
+                                     ctl.bar(L::bFull + s), p * 64, head, (n >> 1) * BN);
+                last[s] = n;
             }
             // drain: every copy this CTA issued lands before its smem is released
             ptx::mbar_wait(ctl.bar(L::bQFull), 0, kWaitLimit);
-            for (int s = 0; s < kStages; ++s) {
-                if (lastK[s] >= 0) ptx::mbar_wait(ctl.bar(L::bKFull + s), (lastK[s] / kStages) & 1, kWaitLimit);
-                if (lastV[s] >= 0) ptx::mbar_wait(ctl.bar(L::bVFull + s), (lastV[s] / kStages) & 1, kWaitLimit);
-            }
+            for (int s = 0; s < kSlots; ++s)
+                if (last[s] >= 0) ptx::mbar_wait(ctl.bar(L::bFull + s), (last[s] / kSlots) & 1, kWaitLimit);
         }
-    } else if (warp == 1) {
+    } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk = ptx::idesc_bf16(BM, BN, false, false);
             constexpr uint32_t idesc_pv = ptx::idesc_bf16(BM, HD, false, true);
-            bool ok = ctl.wait(L::bQFull, 0);
-            auto issue_pv = [&](int i) -> bool {
-                const int st = i % kStages, pb = i & 1;
-                if (!ctl.wait(L::bPFull + pb, (i >> 1) & 1)) return false;
-                if (!ctl.wait(L::bVFull + st, (i / kStages) & 1)) return false;
-                ptx::tc_fence_after();
-                const uint32_t vbase = base + L::kV + st * L::kTile;
-                const uint32_t ptm = tmem + (pb ? L::tP1 : L::tP0);
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t bd = ptx::smem_desc_sw128(vbase + kk * 2048, kPanel, 1024);
-                    ptx::mma_ts(tmem + L::tO, ptm + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
-                }
-                ptx::mma_commit(ctl.bar(L::bVEmpty + st));
-                ptx::mma_commit(ctl.bar(L::bPVDone + pb));
-                return true;
-            };
-            for (int j = 0; ok && j < nt; ++j) {
-                const int st = j % kStages, sb = j & 1;
-                if (!ctl.wait(L::bKFull + st, (j / kStages) & 1)) { ok = false; break; }
-                if (!ctl.wait(L::bSFree + sb, ((j >> 1) & 1) ^ 1)) { ok = false; break; }
-                ptx::tc_fence_after();
-                const uint32_t kbase = base + L::kK + st * L::kTile;
-                const uint32_t stm = tmem + (sb ? L::tS1 : L::tS0);
+            auto slot_of = [](int n) { return n % kSlots; };
+            auto wait_full = [&](int n) { return ctl.wait(L::bFull + slot_of(n), (n / kSlots) & 1); };
+            auto qk = [&](int i, int n) {          // S_i = Q_i K^T, K in load n's slot
+                const uint32_t kb = base + L::kRing + slot_of(n) * L::kTile;
+                const uint32_t qb = base + (i ? L::kQ1 : L::kQ0);
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-                    const uint64_t ad = ptx::smem_desc_sw128(base + L::kQ + off, 16, 1024);
-                    const uint64_t bd = ptx::smem_desc_sw128(kbase + off, 16, 1024);
-                    ptx::mma_ss(stm, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    ptx::mma_ss(tmem + L::tS(i), ptx::smem_desc_sw128(qb + off, 16, 1024),
+                                ptx::smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
                 }
-                ptx::mma_commit(ctl.bar(L::bSFull + sb));
-                ptx::mma_commit(ctl.bar(L::bKEmpty + st));
-                if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+            };
+            auto pv = [&](int i, int n, bool acc) {   // O_i += P_i V, V in load n's slot
+                const uint32_t vb = base + L::kRing + slot_of(n) * L::kTile;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    ptx::mma_ts(tmem + L::tO(i), tmem + L::tS(i) + L::tP + kk * 8,
+                                ptx::smem_desc_sw128(vb + kk * 2048, kPanel, 1024), idesc_pv,
+                                (acc || kk > 0) ? 1u : 0u);
+            };
+            bool ok = ctl.wait(L::bQFull, 0) && wait_full(0);
+            if (ok) {
+                ptx::tc_fence_after();
+                qk(0, 0);
+                ptx::mma_commit(ctl.bar(L::bSFull + 0));
+                qk(1, 0);
+                ptx::mma_commit(ctl.bar(L::bSFull + 1));
+                ptx::mma_commit(ctl.bar(L::bEmpty + slot_of(0)));
             }
-            if (ok) issue_pv(nt - 1);
+            for (int j = 1; ok && j < nt; ++j) {
+                const int nk = 2 * j, nv = 2 * j - 1;        // loads of K_j and V_{j-1}
+                if (!wait_full(nv) || !wait_full(nk)) { ok = false; break; }
+                if (!ctl.wait(L::bPFull + 0, (j - 1) & 1)) { ok = false; break; }
+                ptx::tc_fence_after();
+                pv(0, nv, j > 1);
+                qk(0, nk);
+                ptx::mma_commit(ctl.bar(L::bSFull + 0));
+                if (!ctl.wait(L::bPFull + 1, (j - 1) & 1)) { ok = false; break; }
+                ptx::tc_fence_after();
+                pv(1, nv, j > 1);
+                ptx::mma_commit(ctl.bar(L::bEmpty + slot_of(nv)));
+                qk(1, nk);
+                ptx::mma_commit(ctl.bar(L::bSFull + 1));
+                ptx::mma_commit(ctl.bar(L::bEmpty + slot_of(nk)));
+            }
+            if (ok) {
+                const int nv = 2 * nt - 1;
+                ok = wait_full(nv) && ctl.wait(L::bPFull + 0, (nt - 1) & 1);
+                if (ok) {
+                    ptx::tc_fence_after();
+                    pv(0, nv, nt > 1);
+                    ptx::mma_commit(ctl.bar(L::bOFull + 0));
+                    ok = ctl.wait(L::bPFull + 1, (nt - 1) & 1);
+                }
+                if (ok) {
+                    ptx::tc_fence_after();
+                    pv(1, nv, nt > 1);
+                    ptx::mma_commit(ctl.bar(L::bOFull + 1));
+                    ptx::mma_commit(ctl.bar(L::bEmpty + slot_of(nv)));
+                }
+            }
             // all MMAs of this CTA complete before TMEM can be released
             ptx::mma_commit(ctl.bar(L::bFinal));
             ptx::mbar_wait(ctl.bar(L::bFinal), 0, kWaitLimit);
         }
-    } else {
-        // ------------------------------------------------------------ softmax
+    } else if (warp < 8) {
+        // ------------------------------------------------------------ softmax WG i
+        const int i = warp >> 2;                      // query tile of this warpgroup
         const int q = warp & 3;                       // TMEM lane quarter of this warp
         const int row = q * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        const int qi = q0 + row;
+        const uint32_t tS = tmem + lane_off + L::tS(i);
+        const uint32_t tO = tmem + lane_off + L::tO(i);
+        const int qi = q0 + i * BM + row;
         int t_out = -1;
         if (qi < n_act) {
             t_out = __ldg(idx + qi);
@@ -250,89 +359,25 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         const int tail = n_tokens - (nt - 1) * BN;    // valid keys in the last tile
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
-            const int sb = j & 1;
-            if (!ctl.warp_wait(L::bSFull + sb, (j >> 1) & 1)) { ok = false; break; }
+            if (!ctl.warp_wait(L::bSFull + i, j & 1)) { ok = false; break; }
             ptx::tc_fence_after();
-            const uint32_t stm = tmem + lane_off + (sb ? L::tS1 : L::tS0);
-            uint32_t s[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) ptx::tmem_ld32(stm + 32 * c, s[c]);
-            ptx::tmem_wait_ld();
+            if (j < nt - 1 || tail == BN)
+                softmax_tile<HD, false>(tS, tO, tS + L::tP, j, BN, scale_log2, m, l);
+            else
+                softmax_tile<HD, true>(tS, tO, tS + L::tP, j, tail, scale_log2, m, l);
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(ctl.bar(L::bSFree + sb));
-
-            if (j == nt - 1 && tail < BN) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (32 * c + e >= tail) s[c][e] = __float_as_uint(-INFINITY);
-            }
-            float mx = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-                for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(s[c][e]));
-            const float mxs = mx * scale_log2;
-            // lazy rescale, decided per warp so the TMEM accesses stay warp-wide:
-            // lanes whose max did not grow past 2^8 keep their max (alpha = 1)
-            const bool want = mxs > m + 8.0f;
-            if (__any_sync(0xFFFFFFFFu, want)) {
-                const float m_new = want ? mxs : m;
-                if (j > 0) {
-                    const float alpha = ptx::ex2(m - m_new);
-                    l *= alpha;
-                    // O holds PV_0..PV_{j-1}: wait for the last one, rescale in TMEM
-                    if (!ctl.warp_wait(L::bPVDone + ((j - 1) & 1), ((j - 1) >> 1) & 1)) { ok = false; break; }
-                    ptx::tc_fence_after();
-#pragma unroll
-                    for (int c = 0; c < HD / 32; ++c) {
-                        uint32_t o[32];
-                        ptx::tmem_ld32(tmem + lane_off + L::tO + 32 * c, o);
-                        ptx::tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        ptx::tmem_st32(tmem + lane_off + L::tO + 32 * c, o);
-                    }
-                    ptx::tmem_wait_st();
-                }
-                m = m_new;
-            }
-            uint32_t p[64];
-            float ls = 0.f;
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float a = ptx::ex2(fmaf(__uint_as_float(s[c][e]), scale_log2, -m));
-                    const float b = ptx::ex2(fmaf(__uint_as_float(s[c][e + 1]), scale_log2, -m));
-                    ls += a + b;
-                    p[c * 16 + e / 2] = ptx::pack_bf16(a, b);
-                }
-            l += ls;
-            // P buffer sb was last read by PV_{j-2}
-            if (j >= 2 && !ctl.warp_wait(L::bPVDone + sb, ((j - 2) >> 1) & 1)) { ok = false; break; }
-            ptx::tc_fence_after();
-            const uint32_t ptm = tmem + lane_off + (sb ? L::tP1 : L::tP0);
-            ptx::tmem_st16(ptm, p);
-            ptx::tmem_st16(ptm + 16, p + 16);
-            ptx::tmem_st16(ptm + 32, p + 32);
-            ptx::tmem_st16(ptm + 48, p + 48);
-            ptx::tmem_wait_st();
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(ctl.bar(L::bPFull + sb));
+            if (lane == 0) ptx::mbar_arrive(ctl.bar(L::bPFull + i));
         }
         // ------------------------------------------------------------ epilogue
-        if (ok && ctl.warp_wait(L::bPVDone + ((nt - 1) & 1), ((nt - 1) >> 1) & 1)) {
+        if (ok && ctl.warp_wait(L::bOFull + i, 0)) {
             ptx::tc_fence_after();
             const float inv = 1.0f / l;
             __nv_bfloat16* orow = out + ((size_t)(t_out < 0 ? 0 : t_out) * heads + head) * HD;
 #pragma unroll
             for (int c = 0; c < HD / 32; ++c) {
                 uint32_t o[32];
-                ptx::tmem_ld32(tmem + lane_off + L::tO + 32 * c, o);
+                ptx::tmem_ld32(tO + 32 * c, o);
                 ptx::tmem_wait_ld();
                 uint32_t pk[16];
 #pragma unroll
@@ -351,7 +396,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    if (warp == 1) ptx::tmem_dealloc(tmem, 512);
+    if (warp == 9) ptx::tmem_dealloc(tmem, 512);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -395,7 +440,8 @@ cudaError_t launch_hd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
         if (e != cudaSuccess) return e;
         if (dev < 64) done_mask |= 1ull << dev;
     }
-    const dim3 grid((n_act + BM - 1) / BM, heads);
+    const int q_tiles = (n_act + BM - 1) / BM;
+    const dim3 grid((q_tiles + 1) / 2, heads);
     const float scale_log2 = scale * 1.4426950408889634f;
     attention_kernel<HD><<<grid, kThreads, L::kAlloc, st>>>(
         mq, mk, mv, idx, n_act, n_tokens, heads, scale_log2,
