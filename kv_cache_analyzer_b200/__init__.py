@@ -29,7 +29,9 @@ __all__ = [
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-library_path = os.path.join(_HERE, "libjano.so")
+# JANO_LIBRARY may point at another build of the same library (e.g. a
+# variant compiled with different tuning macros).
+library_path = os.environ.get("JANO_LIBRARY") or os.path.join(_HERE, "libjano.so")
 
 STATUS_NAMES = {0: "JANO_OK", 1: "JANO_EINVAL", 2: "JANO_ESHAPE", 3: "JANO_EALIGN",
                 4: "JANO_EUNSUPPORTED", 5: "JANO_ENONFINITE", 6: "JANO_EINDEX",

@@ -115,34 +115,87 @@ __device__ __forceinline__ void ld64(uint32_t taddr, uint32_t (&r)[64]) {
     ptx::tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
 }
 
-// Row max of 64 values (8 independent chains); with kMask, keys >= valid
-// (the ragged last key tile) are left out.
+// Row max of 64 values (8 independent chains of 3-input max); with kMask,
+// keys >= valid (the ragged last key tile) are left out.
 template <bool kMask>
 __device__ __forceinline__ float max64(const uint32_t (&s)[64], int valid) {
     float m[8];
 #pragma unroll
     for (int a = 0; a < 8; ++a) m[a] = -INFINITY;
 #pragma unroll
-    for (int e = 0; e < 64; ++e)
-        if (!kMask || e < valid) m[e & 7] = fmaxf(m[e & 7], __uint_as_float(s[e]));
-    return fmaxf(fmax4(m[0], m[1], m[2], m[3]), fmax4(m[4], m[5], m[6], m[7]));
+    for (int e = 0; e < 64; e += 2) {
+        float x = __uint_as_float(s[e]), y = __uint_as_float(s[e + 1]);
+        if (kMask && e >= valid) x = -INFINITY;
+        if (kMask && e + 1 >= valid) y = -INFINITY;
+        m[(e >> 1) & 7] = ptx::fmax3(m[(e >> 1) & 7], x, y);
+    }
+    return fmaxf(ptx::fmax3(m[0], m[1], m[2]), ptx::fmax3(m[3], m[4], fmaxf(m[5], fmaxf(m[6], m[7]))));
 }
+
+// 2^x for two lanes on the FMA/ALU pipes, to take part of the exponentials
+// off the MUFU unit (which alone would need about as many cycles per key
+// tile as the tensor core).  Range reduction x = j + f with j = rint(x)
+// (added to the exponent bits) and f in [-1/2, 1/2]; 2^f by a cubic whose
+// coefficients were fitted here by Remez exchange for the smallest maximum
+// relative error on [-1/2, 1/2]: 7.5e-5 (2^-13.7) in fp32 Horner form, far
+// below the 2^-8 rounding of the BF16 P it feeds.  Inputs below -125 are
+// clamped so 2^j stays a normal float (such terms are < 2^-125 of the row
+// maximum).
+__device__ __forceinline__ void exp2_poly2(uint64_t x2, float& ya, float& yb) {
+    constexpr float kC0 = 0x1.fff692p-1f, kC1 = 0x1.62f31ap-1f;
+    constexpr float kC2 = 0x1.f0de1ap-3f, kC3 = 0x1.c3f76p-5f;
+    constexpr float kRound = 12582912.0f;            // 1.5 * 2^23
+    float xa, xb;
+    ptx::f2split(x2, xa, xb);
+    x2 = ptx::f2(fmaxf(xa, -125.0f), fmaxf(xb, -125.0f));
+    const uint64_t r2 = ptx::fadd2(x2, ptx::f2(kRound, kRound));     // low bits hold rint(x)
+    const uint64_t t2 = ptx::fadd2(r2, ptx::f2(-kRound, -kRound));
+    const uint64_t f2 = ptx::ffma2(t2, ptx::f2(-1.f, -1.f), x2);      // f = x - rint(x)
+    uint64_t p2 = ptx::ffma2(ptx::f2(kC3, kC3), f2, ptx::f2(kC2, kC2));
+    p2 = ptx::ffma2(p2, f2, ptx::f2(kC1, kC1));
+    p2 = ptx::ffma2(p2, f2, ptx::f2(kC0, kC0));
+    float ra, rb, pa, pb;
+    ptx::f2split(r2, ra, rb);
+    ptx::f2split(p2, pa, pb);
+    const int ja = __float_as_int(ra) - __float_as_int(kRound);
+    const int jb = __float_as_int(rb) - __float_as_int(kRound);
+    ya = __int_as_float(__float_as_int(pa) + (ja << 23));
+    yb = __int_as_float(__float_as_int(pb) + (jb << 23));
+}
+
+// Share of the exponentials computed by exp2_poly2, in eighths: pairs whose
+// index modulo 8 is below this count (0 = all on MUFU, 2 = a quarter).
+#ifndef JANO_EXP2_POLY_EIGHTHS
+#define JANO_EXP2_POLY_EIGHTHS 2
+#endif
 
 // p = 2^(s*c - m) for 64 values, packed to 32 BF16x2 words; returns sum(p).
 template <bool kMask>
 __device__ __forceinline__ float exp64(const uint32_t (&s)[64], int valid, float c, float m,
                                        uint32_t* pk) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint64_t c2 = ptx::f2(c, c), nm2 = ptx::f2(-m, -m);
+    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
     for (int e = 0; e < 64; e += 2) {
-        float a = ptx::ex2(fmaf(__uint_as_float(s[e]), c, -m));
-        float b = ptx::ex2(fmaf(__uint_as_float(s[e + 1]), c, -m));
+        const uint64_t x2 = ptx::ffma2(ptx::f2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), c2, nm2);
+        float a, b;
+        if (((e >> 1) & 7) < JANO_EXP2_POLY_EIGHTHS) {
+            exp2_poly2(x2, a, b);
+        } else {
+            float xa, xb;
+            ptx::f2split(x2, xa, xb);
+            a = ptx::ex2(xa);
+            b = ptx::ex2(xb);
+        }
         if (kMask && e >= valid) a = 0.f;
         if (kMask && e + 1 >= valid) b = 0.f;
-        acc[(e >> 1) & 3] += a + b;
+        acc[(e >> 1) & 3] = ptx::fadd2(acc[(e >> 1) & 3], ptx::f2(a, b));
         pk[e >> 1] = ptx::pack_bf16(a, b);
     }
-    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    const uint64_t t = ptx::fadd2(ptx::fadd2(acc[0], acc[1]), ptx::fadd2(acc[2], acc[3]));
+    float lo, hi;
+    ptx::f2split(t, lo, hi);
+    return lo + hi;
 }
 
 // One key tile of one query row: row max over S (TMEM, two 64-column
@@ -172,8 +225,14 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, uint32_t 
                 uint32_t o[32];
                 ptx::tmem_ld32(tO + 32 * q, o);
                 ptx::tmem_wait_ld();
+                const uint64_t a2 = ptx::f2(alpha, alpha);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                for (int e = 0; e < 32; e += 2) {
+                    float lo, hi;
+                    ptx::f2split(ptx::fmul2(ptx::f2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), lo, hi);
+                    o[e] = __float_as_uint(lo);
+                    o[e + 1] = __float_as_uint(hi);
+                }
                 ptx::tmem_st32(tO + 32 * q, o);
             }
             ptx::tmem_wait_st();
