@@ -4,92 +4,249 @@
 //   S_b = mean over k=1..K-1, c, (f,h,w) in b of
 //         |x_{k+1} - 2x_k + x_{k-1}| + w_t |D_f x_k| + w_s sqrt(D_h x_k^2 + D_w x_k^2)
 //
-// HBM-bound streaming stencil.  A CTA owns one frame-block x one block-row x
-// a width chunk (a whole number of blocks) and every channel.  Thread
-// (cg, r, w4) owns four consecutive latent elements of one (f,h) row and the
-// channels c = cg, cg+CG, ...; for each channel it walks the K+1 snapshots
-// with float4 loads, keeping the (k-1, k, k+1) window in registers.  The
-// f+1 / h+1 neighbours of snapshot k are float4 loads that hit L1/L2 (the
-// neighbouring rows and frames are being streamed by this and adjacent
-// CTAs), the w+1 neighbour of the fourth element is one scalar load.  Per
-// element sums go to shared memory and one thread per block adds them in a
-// fixed order, so scores are deterministic (no atomics).
+// HBM-bound streaming stencil.  The latent history [K+1][C][F][H][W] is cut
+// into work units of one frame-block x one block-row x a chunk of Wc columns
+// (a whole number of blocks).  A persistent grid walks the units; in each
+// CTA one producer thread streams, for every channel of the unit, a stage of
+// two TMA boxes into a shared-memory ring:
+//   A  all K+1 snapshots of the unit's rows plus the h+1 halo row and 4
+//      extra columns (the w+1 neighbours), box (Wc+4, bh+1, bf, 1, K+1);
+//   B  snapshots 1..K-1 of the next frame's rows (the f+1 neighbours of the
+//      block's last frame), box (Wc, bh, 1, 1, K-1).
+// Out-of-range rows, columns and frames arrive zero-filled and are masked
+// in the arithmetic.  All compute threads work on the same stage: thread
+// (k, row, 4 columns) evaluates the stencil at step k from shared memory with
+// 128-bit loads and keeps its sums over the channels in registers, so the
+// ring can run several stages ahead of the arithmetic.  At the end of a unit
+// the per-thread sums are added per block over k, rows and columns in a
+// fixed order (deterministic, no atomics).
+// Every byte of the latent is read from HBM once; neighbour rows and frames
+// come back from L2.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "jano_common.cuh"
 
 namespace jano {
 namespace {
 
+constexpr int kMaxStages = 16;
+// float4 vectors (4 consecutive columns each) per thread and step
+#ifndef JANO_ANALYZER_VEC
+#define JANO_ANALYZER_VEC 1
+#endif
+constexpr int kVec = JANO_ANALYZER_VEC;
+constexpr long long kWaitLimit = 1ll << 31;
+// Unit width in columns (measured best on the large video latent: 80, i.e.
+// two units per 160-column row) and the shared-memory budget per CTA in KB
+// (0: the smallest of 72 / 110 / 220 KB that holds a ring of >= 4 stages;
+// 72 KB gives three CTAs per SM).
+#ifndef JANO_ANALYZER_WC
+#define JANO_ANALYZER_WC 80
+#endif
+#ifndef JANO_ANALYZER_SMEM_KB
+#define JANO_ANALYZER_SMEM_KB 0
+#endif
+
 struct AGeo {
     int K, C, F, H, W;
     int bf, bh, bw;
     int nBh, nBw;
-    int wchunk;       // latent columns per CTA, multiple of 4 and of bw
-    int cg;           // channel groups per CTA
+    int Wc;                // columns per unit, multiple of 4 and of bw
+    int n_wc;              // units along W
+    int n_units;
+    int NP;                // positions per step: rows x Wc/4
+    int NC;                // compute threads: NP x (K-1), rounded up to 32
+    int S;                 // ring stages
+    int stage_bytes;       // per channel stage, 128-byte multiple
+    int bytesA, bytesB;    // TMA transaction bytes of boxes A and B
+    int offB;              // byte offset of box B in a stage (128-aligned)
+    int red_off;           // offset of the reduction area [K-1][R][Wc]
+    int smem;              // dynamic shared memory bytes
+    int LA;                // floats per staged row of box A (Wc + 4)
     float w_t, w_s;
 };
 
 __device__ __forceinline__ float term(float d2, float df, float dh, float dw, float w_t, float w_s) {
-    return fabsf(d2) + w_t * fabsf(df) + w_s * sqrtf(dh * dh + dw * dw);
+    return fabsf(d2) + w_t * fabsf(df) + w_s * ptx::sqrt_approx(fmaf(dh, dh, dw * dw));
+}
+
+// Bounded wait that also gives up as soon as another thread of the CTA has
+// recorded a timeout (abort flag in shared memory).
+__device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, int* err,
+                                             volatile int* abort) {
+    if (ptx::mbar_try_wait_sleep(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (;;) {
+        if (ptx::mbar_try_wait_sleep(bar, parity)) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > kWaitLimit) {
+            *abort = 1;
+            raise_error(err, JANO_ETIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const void* tmap, uint32_t bar,
+                                            int c0, int c1, int c2, int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar),
+          "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4) : "memory");
+}
+
+__device__ __forceinline__ void named_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
 __global__ void __launch_bounds__(1024)
-analyzer_kernel(const float* __restrict__ lat, AGeo g, float* __restrict__ scores) {
-    extern __shared__ float red[];   // [cg][R][wchunk]
+analyzer_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                AGeo g, float* __restrict__ scores, int* err) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = ptx::smem_u32(smem_raw);
+    const uint32_t base = (raw + 127u) & ~127u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    const int S = g.S;
+    const uint32_t bar_full = base + (uint32_t)g.red_off - 16u * S - 16u;   // S full, S empty barriers
+    volatile int* abort = reinterpret_cast<volatile int*>(gbase + g.red_off - 16);
+    auto full = [&](int s) { return bar_full + 8u * s; };
+    auto empty = [&](int s) { return bar_full + 8u * (S + s); };
+    float* red = reinterpret_cast<float*>(gbase + g.red_off);         // [K-1][R][Wc]
     const int R = g.bf * g.bh;
-    const int W4c = g.wchunk >> 2;
-    const int tid = threadIdx.x;
-    const int w4 = tid % W4c;
-    const int r = (tid / W4c) % R;
-    const int cg = tid / (W4c * R);
+    const int n_compute = g.NC;
 
-    const int fb = blockIdx.z, hb = blockIdx.y;
-    const int f0 = fb * g.bf, h0 = hb * g.bh, w0 = blockIdx.x * g.wchunk;
-    const int rows_f = min(g.bf, g.F - f0), rows_h = min(g.bh, g.H - h0);
-    const int fr = r / g.bh, hr = r % g.bh;
-    const int f = f0 + fr, h = h0 + hr, w = w0 + 4 * w4;
-
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    if (fr < rows_f && hr < rows_h && w < g.W) {
-        const size_t plane = (size_t)g.H * g.W;
-        const size_t snap = (size_t)g.C * g.F * plane;
-        const bool has_f = f + 1 < g.F, has_h = h + 1 < g.H, has_w = w + 4 < g.W;
-        for (int c = cg; c < g.C; c += g.cg) {
-            const float* p = lat + ((size_t)c * g.F + f) * plane + (size_t)h * g.W + w;
-            float4 xm = __ldg(reinterpret_cast<const float4*>(p));
-            float4 x0 = __ldg(reinterpret_cast<const float4*>(p + snap));
-            for (int k = 1; k < g.K; ++k) {
-                const float* pk = p + (size_t)k * snap;
-                const float4 xp = __ldg(reinterpret_cast<const float4*>(pk + snap));
-                const float4 nf = has_f ? __ldg(reinterpret_cast<const float4*>(pk + plane)) : x0;
-                const float4 nh = has_h ? __ldg(reinterpret_cast<const float4*>(pk + g.W)) : x0;
-                const float nw = has_w ? __ldg(pk + 4) : x0.w;
-                a0 += term(xp.x - 2.f * x0.x + xm.x, nf.x - x0.x, nh.x - x0.x, x0.y - x0.x, g.w_t, g.w_s);
-                a1 += term(xp.y - 2.f * x0.y + xm.y, nf.y - x0.y, nh.y - x0.y, x0.z - x0.y, g.w_t, g.w_s);
-                a2 += term(xp.z - 2.f * x0.z + xm.z, nf.z - x0.z, nh.z - x0.z, x0.w - x0.z, g.w_t, g.w_s);
-                a3 += term(xp.w - 2.f * x0.w + xm.w, nf.w - x0.w, nh.w - x0.w, nw - x0.w, g.w_t, g.w_s);
-                xm = x0;
-                x0 = xp;
-            }
+    if (threadIdx.x == 0) {
+        ptx::prefetch_tmap(&tmA);
+        ptx::prefetch_tmap(&tmB);
+        for (int s = 0; s < S; ++s) {
+            ptx::mbar_init(full(s), 1);
+            ptx::mbar_init(empty(s), n_compute / 32);
         }
+        *abort = 0;
+        ptx::fence_mbar_init();
     }
-    float* dst = red + ((size_t)cg * R + r) * g.wchunk + 4 * w4;
-    dst[0] = a0; dst[1] = a1; dst[2] = a2; dst[3] = a3;
     __syncthreads();
 
-    const int nb = g.wchunk / g.bw;
-    for (int ob = tid; ob < nb; ob += blockDim.x) {
-        const int ws = w0 + ob * g.bw;
-        if (ws >= g.W) continue;
-        const int cols = min(g.bw, g.W - ws);
-        float s = 0.f;
-        for (int q = 0; q < g.cg; ++q)
-            for (int rr = 0; rr < R; ++rr) {
-                const float* src = red + ((size_t)q * R + rr) * g.wchunk + ob * g.bw;
-                for (int e = 0; e < g.bw; ++e) s += src[e];
+    const int tid = threadIdx.x;
+    if (tid >= n_compute) {
+        // ------------------------------------------------------------ producer
+        if (tid == n_compute) {
+            int last[kMaxStages];                 // phase of the last copy into each slot
+            for (int q = 0; q < S; ++q) last[q] = -1;
+            int slot = 0, phase = 0;              // ring position, advanced incrementally
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < g.n_units; u += gridDim.x) {
+                const int wc = u % g.n_wc;
+                const int hb = (u / g.n_wc) % g.nBh;
+                const int fb = u / (g.n_wc * g.nBh);
+                const int f0 = fb * g.bf, h0 = hb * g.bh, w0 = wc * g.Wc;
+                const bool has_next = f0 + g.bf < g.F;
+                for (int c = 0; c < g.C; ++c) {
+                    if (!bounded_wait(empty(slot), (uint32_t)(phase ^ 1), err, abort)) { ok = false; break; }
+                    const uint32_t dst = base + (uint32_t)slot * g.stage_bytes;
+                    ptx::mbar_arrive_expect_tx(full(slot), g.bytesA + (has_next ? g.bytesB : 0));
+                    tma_load_5d(dst, &tmA, full(slot), w0, h0, f0, c, 0);
+                    if (has_next)
+                        tma_load_5d(dst + g.offB, &tmB, full(slot), w0, h0, f0 + g.bf, c, 1);
+                    last[slot] = phase;
+                    if (++slot == S) { slot = 0; phase ^= 1; }
+                }
             }
-        const float cnt = (float)(g.K - 1) * (float)g.C * (float)(rows_f * rows_h * cols);
-        scores[((size_t)fb * g.nBh + hb) * g.nBw + (ws / g.bw)] = s / cnt;
+            // drain: the copies this CTA issued land before its smem is released
+            for (int q = 0; q < S; ++q)
+                if (last[q] >= 0) ptx::mbar_wait(full(q), (uint32_t)last[q], kWaitLimit);
+        }
+        return;
     }
+
+    // ---------------------------------------------------------------- compute
+    const int lane = tid & 31;
+    const int Wv = g.Wc / (4 * kVec);              // thread columns (kVec float4 each)
+    const int k = 1 + tid / g.NP;                  // step of this thread (1..K-1; >= K: idle)
+    const int pos = tid % g.NP;
+    const int r = pos / Wv, wv = pos % Wv;
+    const int fr = r / g.bh, hr = r % g.bh;
+    const int LA = g.LA;                           // floats per staged row of box A
+    const int rowsA = g.bh + 1;
+    const int wr = 4 * kVec * wv;
+    // float offsets inside a stage, fixed for the whole kernel
+    const int o_x0 = ((k * g.bf + fr) * rowsA + hr) * LA + wr;
+    const int o_xm = o_x0 - g.bf * rowsA * LA;
+    const int o_xp = o_x0 + g.bf * rowsA * LA;
+    const int o_nh = o_x0 + LA;
+    const int o_nf = fr + 1 < g.bf ? o_x0 + rowsA * LA : g.offB / 4 + ((k - 1) * g.bh + hr) * g.Wc + wr;
+    int slot = 0, phase = 0;                       // ring position, advanced incrementally
+    for (int u = blockIdx.x; u < g.n_units; u += gridDim.x) {
+        const int wc = u % g.n_wc;
+        const int hb = (u / g.n_wc) % g.nBh;
+        const int fb = u / (g.n_wc * g.nBh);
+        const int f0 = fb * g.bf, h0 = hb * g.bh, w0 = wc * g.Wc;
+        const int f = f0 + fr, h = h0 + hr, w = w0 + wr;
+        const bool act = k < g.K && f < g.F && h < g.H && w < g.W;
+        const bool has_f = f + 1 < g.F, has_h = h + 1 < g.H;
+        float acc[4 * kVec];
+#pragma unroll
+        for (int e = 0; e < 4 * kVec; ++e) acc[e] = 0.f;
+        for (int c = 0; c < g.C; ++c) {
+            // after a timeout the CTA stops computing but keeps meeting its barriers
+            const bool ready = bounded_wait(full(slot), (uint32_t)phase, err, abort);
+            if (ready && act) {
+                const float* A = reinterpret_cast<const float*>(gbase + (size_t)slot * g.stage_bytes);
+#pragma unroll
+                for (int v = 0; v < kVec; ++v) {
+                    const float4 x0 = *reinterpret_cast<const float4*>(A + o_x0 + 4 * v);
+                    const float4 xm = *reinterpret_cast<const float4*>(A + o_xm + 4 * v);
+                    const float4 xp = *reinterpret_cast<const float4*>(A + o_xp + 4 * v);
+                    const float4 nh = has_h ? *reinterpret_cast<const float4*>(A + o_nh + 4 * v) : x0;
+                    const float4 nf = has_f ? *reinterpret_cast<const float4*>(A + o_nf + 4 * v) : x0;
+                    // w+1 neighbour of the 4th element; zero-filled beyond the tensor, and the
+                    // difference is dropped there (w + 4v + 4 >= W)
+                    const float nx = A[o_x0 + 4 * v + 4];
+                    const float nw = (w + 4 * v + 4 < g.W) ? nx : x0.w;
+                    float* a = acc + 4 * v;
+                    a[0] += term(xp.x - 2.f * x0.x + xm.x, nf.x - x0.x, nh.x - x0.x, x0.y - x0.x, g.w_t, g.w_s);
+                    a[1] += term(xp.y - 2.f * x0.y + xm.y, nf.y - x0.y, nh.y - x0.y, x0.z - x0.y, g.w_t, g.w_s);
+                    a[2] += term(xp.z - 2.f * x0.z + xm.z, nf.z - x0.z, nh.z - x0.z, x0.w - x0.z, g.w_t, g.w_s);
+                    a[3] += term(xp.w - 2.f * x0.w + xm.w, nf.w - x0.w, nh.w - x0.w, nw - x0.w, g.w_t, g.w_s);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(empty(slot));
+            if (++slot == S) { slot = 0; phase ^= 1; }
+        }
+        // this thread's sums -> red[k-1][r][wr ..] (zeros where inactive or past W)
+        if (k < g.K) {
+            float* dst = red + ((size_t)(k - 1) * R + r) * g.Wc + wr;
+#pragma unroll
+            for (int e = 0; e < 4 * kVec; ++e) dst[e] = (act && w + e < g.W) ? acc[e] : 0.f;
+        }
+        named_sync(1, n_compute);
+        const int nb = g.Wc / g.bw;
+        for (int ob = tid; ob < nb; ob += n_compute) {
+            const int ws = w0 + ob * g.bw;
+            if (ws >= g.W) continue;
+            const int cols = min(g.bw, g.W - ws);
+            const int rows_f = min(g.bf, g.F - f0), rows_h = min(g.bh, g.H - h0);
+            float sum = 0.f;
+            for (int kk = 0; kk < g.K - 1; ++kk)
+                for (int rr = 0; rr < R; ++rr) {
+                    const float* src = red + ((size_t)kk * R + rr) * g.Wc + ob * g.bw;
+                    for (int e = 0; e < g.bw; ++e) sum += src[e];
+                }
+            const float cnt = (float)(g.K - 1) * (float)g.C * (float)(rows_f * rows_h * cols);
+            scores[((size_t)fb * g.nBh + hb) * g.nBw + (ws / g.bw)] = sum / cnt;
+        }
+        named_sync(1, n_compute);
+    }
+}
+
+int gcd(int a, int b) {
+    while (b) { const int t = a % b; a = b; b = t; }
+    return a;
 }
 
 int lcm4(int b) {
@@ -98,47 +255,118 @@ int lcm4(int b) {
     return 4 / a * b;
 }
 
-}  // namespace
-
-cudaError_t launch_block_scores(const float* lat, int K, int C, const jano_geom& g,
-                                float w_t, float w_s, float* scores, int* err,
-                                cudaStream_t st) {
-    (void)err;
-    AGeo a;
-    a.K = K; a.C = C; a.F = g.F; a.H = g.H; a.W = g.W;
-    a.bf = g.bf; a.bh = g.bh; a.bw = g.bw;
-    a.nBh = (g.H + g.bh - 1) / g.bh;
-    a.nBw = (g.W + g.bw - 1) / g.bw;
-    a.w_t = w_t; a.w_s = w_s;
-    const int R = g.bf * g.bh;
-    const int L = lcm4(g.bw);
-    // width chunk: the whole row when it fits, else the widest multiple of L
-    // that keeps R * chunk/4 <= 256 threads per channel group
-    int wchunk = ((g.W + L - 1) / L) * L;
-    while (R * (wchunk / 4) > 256 && wchunk > L) wchunk = ((wchunk / 2 + L - 1) / L) * L;
-    a.wchunk = wchunk;
-    const int per_cg = R * (wchunk / 4);
-    int cg = 512 / per_cg;
-    if (cg < 1) cg = 1;
-    if (cg > C) cg = C;
-    a.cg = cg;
-    const int threads = cg * per_cg;
-    const size_t smem = sizeof(float) * (size_t)cg * R * wchunk;
-    const dim3 grid((g.W + wchunk - 1) / wchunk, a.nBh, (g.F + g.bf - 1) / g.bf);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(analyzer_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    analyzer_kernel<<<grid, threads, smem, st>>>(lat, a, scores);
-    return cudaGetLastError();
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
 }
 
-// Largest block footprint the analyzer launch supports (one channel group).
-bool analyzer_supported(const jano_geom& g) {
-    const int R = g.bf * g.bh;
-    const int L = lcm4(g.bw);
-    return R * (L / 4) <= 1024 && (size_t)R * L * sizeof(float) <= 200 * 1024;
+// Unit width, ring depth and shared memory for a geometry; false if unsupported.
+bool plan(const jano_geom& gm, int K, int C, AGeo& a) {
+    a.K = K; a.C = C; a.F = gm.F; a.H = gm.H; a.W = gm.W;
+    a.bf = gm.bf; a.bh = gm.bh; a.bw = gm.bw;
+    a.nBh = (gm.H + gm.bh - 1) / gm.bh;
+    a.nBw = (gm.W + gm.bw - 1) / gm.bw;
+    const int R = gm.bf * gm.bh;
+    const int L0 = lcm4(gm.bw);
+    const int L = L0 % (4 * kVec) == 0 ? L0 : (4 * kVec) / gcd(L0, 4 * kVec) * L0;   // lcm(L0, 4 kVec)
+    if (gm.bh + 1 > 256 || gm.bf > 256 || K + 1 > 256) return false;
+    // widest unit (a multiple of L, at most the padded row) whose box fits a
+    // TMA box row and whose threads fit a CTA
+    const int Wr = (gm.W + L - 1) / L * L;
+    int Wc = JANO_ANALYZER_WC > 0 ? JANO_ANALYZER_WC / L * L : Wr;
+    if (Wc > Wr) Wc = Wr;
+    while (Wc > L && (Wc + 4 > 256 || (long long)R * (Wc / (4 * kVec)) * (K - 1) + 32 > 1024)) Wc -= L;
+    if (Wc < L || Wc + 4 > 256 || (long long)R * (Wc / (4 * kVec)) * (K - 1) + 32 > 1024) return false;
+    a.Wc = Wc;
+    a.LA = Wc + 4;
+    a.n_wc = (gm.W + Wc - 1) / Wc;
+    a.n_units = ((gm.F + gm.bf - 1) / gm.bf) * a.nBh * a.n_wc;
+    a.NP = R * (Wc / (4 * kVec));
+    a.NC = (a.NP * (K - 1) + 31) / 32 * 32;
+    a.bytesA = a.LA * (gm.bh + 1) * gm.bf * (K + 1) * 4;
+    a.bytesB = Wc * gm.bh * (K - 1) * 4;
+    a.offB = (a.bytesA + 127) / 128 * 128;
+    a.stage_bytes = (a.offB + a.bytesB + 127) / 128 * 128;
+    const long long fixed = (long long)(K - 1) * R * Wc * 4 + 128 + 16;   // red + slack + abort
+    auto stages_for = [&](long long budget) {
+        long long n = (budget - fixed) / (a.stage_bytes + 16);
+        return n > kMaxStages ? kMaxStages : n;
+    };
+    long long budget = JANO_ANALYZER_SMEM_KB * 1024ll;
+    if (JANO_ANALYZER_SMEM_KB == 0) {
+        budget = 220 * 1024ll;
+        for (long long b : {72 * 1024ll, 110 * 1024ll})
+            if (stages_for(b) >= 4) { budget = b; break; }
+    }
+    const long long S = stages_for(budget);
+    if (S < 2) return false;
+    a.S = (int)S;
+    a.red_off = a.S * a.stage_bytes + 16 * a.S + 16;     // barriers and abort flag sit below red
+    a.smem = a.red_off + (K - 1) * R * Wc * 4 + 128;
+    return true;
+}
+
+}  // namespace
+
+bool analyzer_supported(const jano_geom& g, int K, int C) {
+    AGeo a;
+    return plan(g, K, C, a);
+}
+
+cudaError_t launch_block_scores(const float* lat, int K, int C, const jano_geom& gm,
+                                float w_t, float w_s, float* scores, int* err,
+                                cudaStream_t st) {
+    AGeo a;
+    if (!plan(gm, K, C, a)) return cudaErrorInvalidValue;
+    a.w_t = w_t;
+    a.w_s = w_s;
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorInvalidValue;
+    const cuuint64_t dims[5] = {(cuuint64_t)gm.W, (cuuint64_t)gm.H, (cuuint64_t)gm.F, (cuuint64_t)C,
+                                (cuuint64_t)(K + 1)};
+    const cuuint64_t strides[4] = {(cuuint64_t)gm.W * 4, (cuuint64_t)gm.H * gm.W * 4,
+                                   (cuuint64_t)gm.F * gm.H * gm.W * 4,
+                                   (cuuint64_t)C * gm.F * gm.H * gm.W * 4};
+    const cuuint32_t boxA[5] = {(cuuint32_t)a.Wc + 4, (cuuint32_t)gm.bh + 1, (cuuint32_t)gm.bf, 1,
+                                (cuuint32_t)K + 1};
+    const cuuint32_t boxB[5] = {(cuuint32_t)a.Wc, (cuuint32_t)gm.bh, 1, 1, (cuuint32_t)K - 1};
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    CUtensorMap mA, mB;
+    if (fn(&mA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, const_cast<float*>(lat), dims, strides, boxA, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        fn(&mB, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, const_cast<float*>(lat), dims, strides, boxB, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+
+    const size_t smem = (size_t)a.smem;
+    static unsigned long long done_mask = 0;   // per-device shared-memory opt-in
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (dev >= 64 || !(done_mask & (1ull << dev))) {
+        cudaError_t e = cudaFuncSetAttribute(analyzer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             224 * 1024);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) done_mask |= 1ull << dev;
+    }
+    const int threads = a.NC + 32;
+    // resident CTAs per SM: shared memory (228 KB, 1 KB reserved per CTA) and threads
+    int per_sm = (228 * 1024) / (a.smem + 1024);
+    if (per_sm > 2048 / threads) per_sm = 2048 / threads;
+    if (per_sm < 1) per_sm = 1;
+    const int grid = a.n_units < per_sm * sms ? a.n_units : per_sm * sms;
+    analyzer_kernel<<<grid, threads, smem, st>>>(mA, mB, a, scores, err);
+    return cudaGetLastError();
 }
 
 }  // namespace jano

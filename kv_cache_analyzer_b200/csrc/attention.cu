@@ -105,10 +105,6 @@ struct Ctl {
     }
 };
 
-__device__ __forceinline__ float fmax4(float a, float b, float c, float d) {
-    return fmaxf(fmaxf(a, b), fmaxf(c, d));
-}
-
 // 64 consecutive TMEM columns of this warp's 32 lanes into registers.
 __device__ __forceinline__ void ld64(uint32_t taddr, uint32_t (&r)[64]) {
     ptx::tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));

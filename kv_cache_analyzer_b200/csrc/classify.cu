@@ -4,153 +4,196 @@
 //
 // Blocks are ranked by the key (score, block index).  A block is Static when
 // its rank is below k_static = n_S and Active when its rank is at least
-// k_active = n - n_A.  Instead of sorting, one thread block finds, for each
-// of the two rank thresholds, the 32-bit score key sitting at that rank with
-// an MSB-first radix select (4 passes of 8-bit digits, shared-memory
-// histograms), then one pass in index order resolves ties at the threshold
-// value with a block-wide ballot scan: among equal scores the lower block
-// index ranks lower.  Exact and deterministic; no scratch memory.  The n
-// scores are re-read from L2 on each pass (n is at most a few 10^5).
+// k_active = n - n_A.  Instead of sorting, the kernel finds, for each of the
+// two rank thresholds, the 32-bit order-preserving score key at that rank by
+// an MSB-first radix select (digits of 11, 11 and 10 bits), then resolves
+// ties at the threshold value by block index in one pass in index order.
+//
+// One thread-block cluster of 8 CTAs does the work with no global scratch:
+// each CTA histograms its eighth of the scores in shared memory (warp-
+// aggregated atomics, since most keys share their top digits), the 8
+// histograms are summed through distributed shared memory after a cluster
+// barrier, and every CTA picks the same digit.  Histograms are double
+// buffered so one cluster barrier per pass suffices.  The tie pass counts
+// threshold ties per thread over a contiguous range, scans them inside the
+// CTA and across the 8 CTAs (again through distributed shared memory), then
+// writes the levels.  Exact and deterministic.
+#include <cooperative_groups.h>
+
 #include "jano_common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace jano {
 namespace {
 
+constexpr int kCluster = 8;
 constexpr int kThreads = 1024;
-constexpr int kChunk = 8;    // independent loads in flight per thread
+constexpr int kBins = 2048;             // 11-bit digits
+constexpr int kPasses = 3;
+__host__ __device__ constexpr int digit_shift(int pass) { return pass == 0 ? 21 : (pass == 1 ? 10 : 0); }
+__host__ __device__ constexpr int digit_width(int pass) { return pass == 2 ? 10 : 11; }
 
-// Order-preserving map float -> uint32 (unsigned order == float order),
+// Order-preserving map float bits -> uint32 (unsigned order == float order),
 // with -0 folded onto +0.
 __device__ __forceinline__ uint32_t order_key(uint32_t b) {
     if (b == 0x80000000u) b = 0u;
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+struct Shared {
+    // [buffer][target][bin], 32 KB.  Pass p histograms into buffer p&1; once
+    // the pass's cluster barrier has passed, no peer reads buffer (p&1)^1 any
+    // more, so it holds this CTA's copy of the cluster-wide totals.
+    unsigned hist[2][2][kBins];
+    unsigned val[2], need[2];            // per target: key prefix, rank left
+    unsigned wsum[2][32];
+    unsigned ctot[2];                    // this CTA's tie counts (read by peers)
+    int bad;
+};
+
+__device__ __forceinline__ void warp_agg_add(unsigned* h, unsigned active, unsigned dg, bool mine) {
+    if (!mine) return;
+    const unsigned peers = __match_any_sync(active, dg);
+    if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[dg], __popc(peers));
+}
+
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
 classify_kernel(const uint32_t* __restrict__ bits, int n, long long k_static,
                 long long k_active, uint8_t* __restrict__ levels, int* err) {
-    __shared__ unsigned hist[2][256];
-    __shared__ unsigned s_val[2];
-    __shared__ unsigned s_need[2];
-    __shared__ unsigned s_wtot[2][32];
+    __shared__ Shared sh;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    // targets: t=0 -> rank k_static, t=1 -> rank k_active; "live" if 0 < k < n
-    const long long ks[2] = {k_static, k_active};
+    // this CTA's slice of the scores
+    const int per_cta = (n + kCluster - 1) / kCluster;
+    const int lo = min(n, rank * per_cta), hi = min(n, lo + per_cta);
+
     const bool live0 = k_static > 0 && k_static < n;
     const bool live1 = k_active > 0 && k_active < n;
 
-    // ---- pass 0: reject non-finite scores -----------------------------------
+    // ---- non-finite scores: any CTA seeing one makes the whole cluster stop
     int bad = 0;
-    for (int base = 0; base < n; base += kThreads * kChunk) {
-        uint32_t v[kChunk];
-#pragma unroll
-        for (int j = 0; j < kChunk; ++j) {
-            const int i = base + j * kThreads + tid;
-            v[j] = i < n ? __ldg(bits + i) : 0u;
-        }
-#pragma unroll
-        for (int j = 0; j < kChunk; ++j) bad |= (v[j] & 0x7F800000u) == 0x7F800000u;
+    for (int i = lo + tid; i < hi; i += kThreads)
+        bad |= (__ldg(bits + i) & 0x7F800000u) == 0x7F800000u;
+    bad = __syncthreads_or(bad);
+    if (tid == 0) {
+        sh.bad = bad;
+        sh.val[0] = sh.val[1] = 0u;
+        sh.need[0] = (unsigned)(k_static < 0 ? 0 : (k_static > n ? n : k_static));
+        sh.need[1] = (unsigned)(k_active < 0 ? 0 : (k_active > n ? n : k_active));
     }
-    if (__syncthreads_or(bad)) {
-        if (tid == 0) raise_error(err, JANO_ENONFINITE);
+    cluster.sync();
+    int any_bad = 0;
+    for (int r = 0; r < kCluster; ++r) any_bad |= *cluster.map_shared_rank(&sh.bad, r);
+    if (any_bad) {
+        if (rank == 0 && tid == 0) raise_error(err, JANO_ENONFINITE);
+        cluster.sync();            // peers may still be reading our flag
         return;
     }
 
-    if (tid < 2) {
-        s_val[tid] = 0u;
-        s_need[tid] = (unsigned)(ks[tid] < 0 ? 0 : (ks[tid] > n ? n : ks[tid]));
-    }
-
-    // ---- radix select, most significant digit first -------------------------
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
-        for (int b = tid; b < 512; b += kThreads) (&hist[0][0])[b] = 0u;
+    // ---- radix select, most significant digit first
+    for (int pass = 0; pass < kPasses; ++pass) {
+        const int buf = pass & 1, shift = digit_shift(pass);
+        const unsigned dmask = (1u << digit_width(pass)) - 1u;
+        const uint32_t hmask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + digit_width(pass)));
+        for (int b = tid; b < 2 * kBins; b += kThreads) (&sh.hist[buf][0][0])[b] = 0u;
         __syncthreads();
-        const uint32_t p0 = s_val[0] & hi_mask, p1 = s_val[1] & hi_mask;
-        for (int base = 0; base < n; base += kThreads * kChunk) {
-            uint32_t v[kChunk];
-#pragma unroll
-            for (int j = 0; j < kChunk; ++j) {
-                const int i = base + j * kThreads + tid;
-                v[j] = i < n ? order_key(__ldg(bits + i)) : 0u;
-            }
-#pragma unroll
-            for (int j = 0; j < kChunk; ++j) {
-                if (base + j * kThreads + tid < n) {
-                    const uint32_t dg = (v[j] >> shift) & 0xFFu;
-                    if (live0 && (v[j] & hi_mask) == p0) atomicAdd(&hist[0][dg], 1u);
-                    if (live1 && (v[j] & hi_mask) == p1) atomicAdd(&hist[1][dg], 1u);
-                }
-            }
+        const uint32_t p0 = sh.val[0] & hmask, p1 = sh.val[1] & hmask;
+        for (int base = lo; base < hi; base += kThreads) {
+            const int i = base + tid;
+            const bool ok = i < hi;
+            const uint32_t u = ok ? order_key(__ldg(bits + i)) : 0u;
+            const unsigned dg = (u >> shift) & dmask;
+            const bool m0 = ok && live0 && (u & hmask) == p0;
+            const bool m1 = ok && live1 && (u & hmask) == p1;
+            const unsigned a0 = __ballot_sync(0xFFFFFFFFu, m0);
+            const unsigned a1 = __ballot_sync(0xFFFFFFFFu, m1);
+            warp_agg_add(sh.hist[buf][0], a0, dg, m0);
+            warp_agg_add(sh.hist[buf][1], a1, dg, m1);
+        }
+        cluster.sync();            // all 8 local histograms of this pass are complete
+        for (int b = tid; b < 2 * kBins; b += kThreads) {
+            unsigned s = 0;
+            for (int r = 0; r < kCluster; ++r)
+                s += cluster.map_shared_rank(&sh.hist[buf][0][0], r)[b];
+            (&sh.hist[buf ^ 1][0][0])[b] = s;
         }
         __syncthreads();
         if (warp < 2 && (warp == 0 ? live0 : live1)) {
-            // lane owns bins [8*lane, 8*lane+8)
-            unsigned c[8], s = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) { c[j] = hist[warp][8 * lane + j]; s += c[j]; }
+            // lane owns 64 consecutive bins
+            const unsigned* t = sh.hist[buf ^ 1][warp] + 64 * lane;
+            unsigned s = 0;
+            for (int j = 0; j < 64; ++j) s += t[j];
             unsigned incl = s;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const unsigned y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
                 if (lane >= o) incl += y;
             }
-            const unsigned need = s_need[warp];
+            const unsigned need = sh.need[warp];
             const unsigned excl = incl - s;
-            // the lane whose range holds the need-th candidate (0-based)
-            const bool mine = excl <= need && need < incl;
-            if (mine) {
+            if (excl <= need && need < incl) {
                 unsigned acc = excl;
-                int dg = 8 * lane;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (acc + c[j] > need) { dg = 8 * lane + j; break; }
-                    acc += c[j];
+                int dg = 64 * lane;
+                for (int j = 0; j < 64; ++j) {
+                    if (acc + t[j] > need) { dg = 64 * lane + j; break; }
+                    acc += t[j];
                 }
-                s_val[warp] |= (uint32_t)dg << shift;
-                s_need[warp] = need - acc;
+                sh.val[warp] |= (uint32_t)dg << shift;
+                sh.need[warp] = need - acc;
             }
         }
         __syncthreads();
     }
 
-    // ---- final pass: ties at the threshold value resolved by block index ----
-    const uint32_t v0 = s_val[0], v1 = s_val[1];
-    const unsigned need0 = s_need[0], need1 = s_need[1];
-    unsigned run0 = 0, run1 = 0;
-    const unsigned lt_mask = (1u << lane) - 1u;
-    for (int base = 0; base < n; base += kThreads) {
-        const int i = base + tid;
-        const bool ok = i < n;
-        const uint32_t u = ok ? order_key(__ldg(bits + i)) : 0u;
-        const bool e0 = ok && live0 && u == v0;
-        const bool e1 = ok && live1 && u == v1;
-        const unsigned b0 = __ballot_sync(0xFFFFFFFFu, e0);
-        const unsigned b1 = __ballot_sync(0xFFFFFFFFu, e1);
-        if (lane == 0) { s_wtot[0][warp] = __popc(b0); s_wtot[1][warp] = __popc(b1); }
-        __syncthreads();
-        unsigned pre0 = 0, pre1 = 0, tot0 = 0, tot1 = 0;
-        for (int w = 0; w < kThreads / 32; ++w) {
-            const unsigned a0 = s_wtot[0][w], a1 = s_wtot[1][w];
-            if (w < warp) { pre0 += a0; pre1 += a1; }
-            tot0 += a0;
-            tot1 += a1;
-        }
-        if (ok) {
-            const unsigned tie0 = run0 + pre0 + __popc(b0 & lt_mask);
-            const unsigned tie1 = run1 + pre1 + __popc(b1 & lt_mask);
-            // rank < k_static ?
-            const bool below_s = live0 ? (u < v0 || (e0 && tie0 < need0)) : (k_static >= n);
-            // rank < k_active ?
-            const bool below_a = live1 ? (u < v1 || (e1 && tie1 < need1)) : (k_active >= n);
-            levels[i] = below_s ? 1 : (below_a ? 2 : 3);
-        }
-        run0 += tot0;
-        run1 += tot1;
-        __syncthreads();
+    // ---- ties at the threshold values, resolved by block index
+    const uint32_t v0 = sh.val[0], v1 = sh.val[1];
+    const unsigned need0 = sh.need[0], need1 = sh.need[1];
+    const int per_thr = (hi - lo + kThreads - 1) / kThreads;
+    const int tlo = min(hi, lo + tid * per_thr), thi = min(hi, tlo + per_thr);
+    unsigned c0 = 0, c1 = 0;
+    for (int i = tlo; i < thi; ++i) {
+        const uint32_t u = order_key(__ldg(bits + i));
+        c0 += live0 && u == v0;
+        c1 += live1 && u == v1;
     }
+    // exclusive scan of (c0, c1) over the CTA's threads
+    unsigned s0 = c0, s1 = c1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y0 = __shfl_up_sync(0xFFFFFFFFu, s0, o);
+        const unsigned y1 = __shfl_up_sync(0xFFFFFFFFu, s1, o);
+        if (lane >= o) { s0 += y0; s1 += y1; }
+    }
+    if (lane == 31) { sh.wsum[0][warp] = s0; sh.wsum[1][warp] = s1; }
+    __syncthreads();
+    unsigned w0 = 0, w1 = 0, t0 = 0, t1 = 0;
+    for (int w = 0; w < kThreads / 32; ++w) {
+        if (w < warp) { w0 += sh.wsum[0][w]; w1 += sh.wsum[1][w]; }
+        t0 += sh.wsum[0][w];
+        t1 += sh.wsum[1][w];
+    }
+    if (tid == 0) { sh.ctot[0] = t0; sh.ctot[1] = t1; }
+    cluster.sync();
+    unsigned b0 = 0, b1 = 0;
+    for (int r = 0; r < rank; ++r) {
+        b0 += cluster.map_shared_rank(sh.ctot, r)[0];
+        b1 += cluster.map_shared_rank(sh.ctot, r)[1];
+    }
+    unsigned tie0 = b0 + w0 + s0 - c0, tie1 = b1 + w1 + s1 - c1;
+    for (int i = tlo; i < thi; ++i) {
+        const uint32_t u = order_key(__ldg(bits + i));
+        const bool e0 = live0 && u == v0, e1 = live1 && u == v1;
+        // rank < k_static ?  rank < k_active ?
+        const bool below_s = live0 ? (u < v0 || (e0 && tie0 < need0)) : (k_static >= n);
+        const bool below_a = live1 ? (u < v1 || (e1 && tie1 < need1)) : (k_active >= n);
+        levels[i] = below_s ? 1 : (below_a ? 2 : 3);
+        tie0 += e0;
+        tie1 += e1;
+    }
+    cluster.sync();                // keep shared memory alive until peers are done
 }
 
 }  // namespace
@@ -158,8 +201,8 @@ classify_kernel(const uint32_t* __restrict__ bits, int n, long long k_static,
 cudaError_t launch_classify(const float* scores, int n, long long k_static,
                             long long k_active, uint8_t* levels, int* err,
                             cudaStream_t st) {
-    classify_kernel<<<1, kThreads, 0, st>>>(reinterpret_cast<const uint32_t*>(scores), n,
-                                            k_static, k_active, levels, err);
+    classify_kernel<<<kCluster, kThreads, 0, st>>>(reinterpret_cast<const uint32_t*>(scores), n,
+                                                   k_static, k_active, levels, err);
     return cudaGetLastError();
 }
 

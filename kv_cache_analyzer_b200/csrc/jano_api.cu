@@ -62,9 +62,7 @@ jano_status jano_block_scores(const float* lat, int K, int C, const jano_geom* g
     if (gs != JANO_OK) return gs;
     if (g->W % 4) return JANO_EUNSUPPORTED;
     if (!aligned16(lat)) return JANO_EALIGN;
-    if (!analyzer_supported(*g)) return JANO_EUNSUPPORTED;
-    if ((long long)g->F > 65535 || (long long)((g->H + g->bh - 1) / g->bh) > 65535)
-        return JANO_EUNSUPPORTED;
+    if (!analyzer_supported(*g, K, C)) return JANO_EUNSUPPORTED;
     int* err = device_error_word();
     if (!err) return JANO_ECUDA;
     return from_cuda(launch_block_scores(lat, K, C, *g, w_temporal, w_spatial, scores, err,

@@ -31,7 +31,7 @@ cudaError_t launch_block_scores(const float* lat, int K, int C, const jano_geom&
 cudaError_t launch_classify(const float* scores, int n, long long k_static,
                             long long k_active, uint8_t* levels, int* err,
                             cudaStream_t st);
-bool analyzer_supported(const jano_geom& g);
+bool analyzer_supported(const jano_geom& g, int K, int C);
 size_t schedule_workspace_bytes(const jano_geom& g);
 cudaError_t launch_build_schedule(const uint8_t* block_levels, const jano_geom& g,
                                   const jano_sched_cfg& c, int32_t* offsets,
@@ -72,6 +72,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
                  "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
                  "selp.u32 %0, 1, 0, p;\n\t}"
                  : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Like mbar_try_wait, but a thread whose phase is not complete is suspended
+// (issues nothing) for up to `hint_ns` nanoseconds instead of returning at
+// once, so many waiting warps do not burn issue slots spinning.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns = 20000) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity), "r"(hint_ns) : "memory");
     return ok != 0;
 }
 
@@ -206,6 +219,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
          | ((b_mn_major ? 1u : 0u) << 16)
          | ((uint32_t)(N >> 3) << 17)
          | ((uint32_t)(M >> 4) << 24);
+}
+
+// Hardware square root approximation (relative error about 2^-22).
+__device__ __forceinline__ float sqrt_approx(float x) {
+    float y;
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 __device__ __forceinline__ float ex2(float x) {

@@ -91,3 +91,22 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch, jl):
     monkeypatch.setattr(jl, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         jl.lib()
+
+
+def test_every_workload_geometry_passes_host_support_checks(jl):
+    # On a machine without a GPU a supported call gets past validation and
+    # fails only at the device lookup (JANO_ECUDA); an unsupported shape
+    # would return JANO_EUNSUPPORTED (4) before that.
+    import synth
+    L = jl.lib()
+    fake = C.c_void_p(256)
+    for name, w in synth.WORKLOADS.items():
+        g = jl.Geometry(w.F, w.H, w.W, w.block, w.patch).c()
+        code = L.jano_block_scores(fake, w.K, w.C, C.byref(g), 0.5, 0.5, fake, None)
+        assert code != 4, name
+    for shape, block in [((3, 2, 3, 9, 12), (1, 4, 4)), ((4, 3, 5, 6, 8), (2, 3, 2)),
+                         ((6, 1, 1, 16, 16), (1, 2, 2)), ((3, 1, 2, 4, 20), (1, 4, 8)),
+                         ((9, 64, 8, 64, 256), (2, 8, 8)), ((6, 16, 1, 720, 1280), (1, 4, 4))]:
+        K1, Cc, F, H, W = shape
+        g = jl.Geometry(F, H, W, block, (1, 1, 1)).c()
+        assert L.jano_block_scores(fake, K1 - 1, Cc, C.byref(g), 0.5, 0.5, fake, None) != 4, shape

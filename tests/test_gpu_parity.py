@@ -70,7 +70,9 @@ def test_block_scores_match_oracle(J, name):
 @pytest.mark.parametrize("shape,block", [((3, 2, 3, 9, 12), (1, 4, 4)),     # partial rows/cols
                                          ((4, 3, 5, 6, 8), (2, 3, 2)),      # bf > 1, odd blocks
                                          ((6, 1, 1, 16, 16), (1, 2, 2)),    # F = 1
-                                         ((3, 1, 2, 4, 20), (1, 4, 8))])    # bw = 8, partial
+                                         ((3, 1, 2, 4, 20), (1, 4, 8)),     # bw = 8, partial
+                                         ((4, 3, 3, 9, 520), (1, 4, 4)),    # wide rows: boxed chunks
+                                         ((3, 2, 2, 6, 200), (2, 4, 8))])   # whole rows, bf = 2
 def test_block_scores_edge_geometries(J, shape, block):
     g = np.random.default_rng(sum(shape))
     lat = g.standard_normal(shape).astype(np.float32)
