@@ -67,6 +67,23 @@ def workload_config(w):
     }
 
 
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(x: float, dist=None, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity without a group);
+    a CUDA tensor for NCCL, a CPU tensor otherwise."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device or "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Aggregate throughput: every rank processes its own replica."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ inputs
 def make_inputs(w, seed_shift=0):
     import synth
@@ -274,13 +291,9 @@ def run_gpu(args, w, rank, world, local_rank, dist):
     stage = np.array([[e[k].elapsed_time(e[k + 1]) for k in range(5)] for e in evs])  # ms
     # stage columns: scores, classify, schedule, scatter, attention
     stage_ms = stage.mean(axis=0)
-    t_max = total_ms
-    if dist is not None:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt.item())
+    t_max = max_over_ranks(total_ms, dist, dev)
     ms_per_step = t_max / args.steps
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tflops(flops, world, ms_per_step)
     code = J.device_error(stream)
     if code:
         raise RuntimeError(f"device error in timed region: {J.jano_status_str(code)}")
@@ -303,12 +316,8 @@ def run_gpu(args, w, rank, world, local_rank, dist):
         e2.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        e2e_ms = s2.elapsed_time(e2)
-        if dist is not None:
-            tt = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
-        e2e = {"value": world * flops / (e2e_ms / args.steps * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e_ms = max_over_ranks(s2.elapsed_time(e2), dist, dev)
+        e2e = {"value": whole_job_tflops(flops, world, e2e_ms / args.steps), "unit": "TFLOP/s",
                "h2d_bytes_per_step": HotPath.h2d_bytes(host),
                "d2h_bytes_per_step": host_out.numel() * host_out.element_size()}
 
