@@ -13,8 +13,10 @@
 //              S (128 fp32) is read from TMEM in two halves, the running max
 //              is kept in the log2 domain and O is rescaled in TMEM only when
 //              the max grows by more than 2^8 (lazy rescale), P is written as
-//              packed BF16 into the upper half of the row's S columns, and at
-//              the end O is normalised and stored as BF16 to out[idx[i]].
+//              packed BF16 into the upper half of the row's S columns (keys
+//              64..127 first, published on their own barrier so their P.V
+//              starts while keys 0..63 are exponentiated), and at the end O
+//              is normalised and stored as BF16 to out[idx[i]].
 //   warp 8     TMA producer: both Q tiles once, then K_j, V_j (128 keys x d)
 //              into a 4-slot shared-memory ring (128-byte swizzle, boxes of
 //              64 columns); completion counted on mbarriers.
@@ -63,8 +65,9 @@ struct Layout {
     static constexpr int bFull = 1;                    // [kSlots]
     static constexpr int bEmpty = bFull + kSlots;      // [kSlots]
     static constexpr int bSFull = bEmpty + kSlots;     // [2]
-    static constexpr int bPFull = bSFull + 2;          // [2]
-    static constexpr int bOFull = bPFull + 2;          // [2]
+    static constexpr int bPFull = bSFull + 2;          // [2] whole P written
+    static constexpr int bPHalf = bPFull + 2;          // [2] P of keys 64..127 written
+    static constexpr int bOFull = bPHalf + 2;          // [2]
     static constexpr int bFinal = bOFull + 2;
     static constexpr int kNumBars = bFinal + 1;
     static constexpr uint32_t kMisc = kBar + 8 * kNumBars;        // tmem base, abort flag
@@ -199,7 +202,7 @@ __device__ __forceinline__ float exp64(const uint32_t (&s)[64], int valid, float
 // the row's S columns.  Warp-uniform control flow throughout.
 template <int HD, bool kMask>
 __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, uint32_t tP, int j, int valid,
-                                             float c, float& m, float& l) {
+                                             float c, float& m, float& l, uint32_t bar_half) {
     uint32_t s[64];
     ld64(tS, s);
     ptx::tmem_wait_ld();
@@ -239,6 +242,12 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, uint32_t 
     uint32_t pk[32];
     l += exp64<kMask>(s, valid - 64, c, m, pk);
     ptx::tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(pk));
+    // hand the upper key half to the MMA thread now: its P.V runs while the
+    // lower half's exponentials are computed
+    ptx::tmem_wait_st();
+    ptx::tc_fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(bar_half);
     ld64(tS, s);
     ptx::tmem_wait_ld();
     l += exp64<kMask>(s, valid, c, m, pk);
@@ -282,6 +291,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(ctl.bar(L::bSFull + s), 1);
             ptx::mbar_init(ctl.bar(L::bPFull + s), 4);
+            ptx::mbar_init(ctl.bar(L::bPHalf + s), 4);
             ptx::mbar_init(ctl.bar(L::bOFull + s), 1);
         }
         ptx::mbar_init(ctl.bar(L::bFinal), 1);
@@ -340,13 +350,24 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
                                 ptx::smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
                 }
             };
-            auto pv = [&](int i, int n, bool acc) {   // O_i += P_i V, V in load n's slot
+            // O_i += P_i V over key sixteenths [k0, k1); V in load n's slot
+            auto pv = [&](int i, int n, int k0, int k1, bool acc) {
                 const uint32_t vb = base + L::kRing + slot_of(n) * L::kTile;
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
+                for (int kk = k0; kk < k1; ++kk)
                     ptx::mma_ts(tmem + L::tO(i), tmem + L::tS(i) + L::tP + kk * 8,
                                 ptx::smem_desc_sw128(vb + kk * 2048, kPanel, 1024), idesc_pv,
-                                (acc || kk > 0) ? 1u : 0u);
+                                (acc || kk > k0) ? 1u : 0u);
+            };
+            // P_i of tile j: upper key half as soon as it is published, then the lower half
+            auto pv_tile = [&](int i, int n, int j) -> bool {
+                if (!ctl.wait(L::bPHalf + i, j & 1)) return false;
+                ptx::tc_fence_after();
+                pv(i, n, BN / 32, BN / 16, j > 0);
+                if (!ctl.wait(L::bPFull + i, j & 1)) return false;
+                ptx::tc_fence_after();
+                pv(i, n, 0, BN / 32, true);
+                return true;
             };
             bool ok = ctl.wait(L::bQFull, 0) && wait_full(0);
             if (ok) {
@@ -360,14 +381,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
             for (int j = 1; ok && j < nt; ++j) {
                 const int nk = 2 * j, nv = 2 * j - 1;        // loads of K_j and V_{j-1}
                 if (!wait_full(nv) || !wait_full(nk)) { ok = false; break; }
-                if (!ctl.wait(L::bPFull + 0, (j - 1) & 1)) { ok = false; break; }
-                ptx::tc_fence_after();
-                pv(0, nv, j > 1);
+                if (!pv_tile(0, nv, j - 1)) { ok = false; break; }
                 qk(0, nk);
                 ptx::mma_commit(ctl.bar(L::bSFull + 0));
-                if (!ctl.wait(L::bPFull + 1, (j - 1) & 1)) { ok = false; break; }
-                ptx::tc_fence_after();
-                pv(1, nv, j > 1);
+                if (!pv_tile(1, nv, j - 1)) { ok = false; break; }
                 ptx::mma_commit(ctl.bar(L::bEmpty + slot_of(nv)));
                 qk(1, nk);
                 ptx::mma_commit(ctl.bar(L::bSFull + 1));
@@ -375,16 +392,12 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
             if (ok) {
                 const int nv = 2 * nt - 1;
-                ok = wait_full(nv) && ctl.wait(L::bPFull + 0, (nt - 1) & 1);
+                ok = wait_full(nv) && pv_tile(0, nv, nt - 1);
                 if (ok) {
-                    ptx::tc_fence_after();
-                    pv(0, nv, nt > 1);
                     ptx::mma_commit(ctl.bar(L::bOFull + 0));
-                    ok = ctl.wait(L::bPFull + 1, (nt - 1) & 1);
+                    ok = pv_tile(1, nv, nt - 1);
                 }
                 if (ok) {
-                    ptx::tc_fence_after();
-                    pv(1, nv, nt > 1);
                     ptx::mma_commit(ctl.bar(L::bOFull + 1));
                     ptx::mma_commit(ctl.bar(L::bEmpty + slot_of(nv)));
                 }
@@ -417,9 +430,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (!ctl.warp_wait(L::bSFull + i, j & 1)) { ok = false; break; }
             ptx::tc_fence_after();
             if (j < nt - 1 || tail == BN)
-                softmax_tile<HD, false>(tS, tO, tS + L::tP, j, BN, scale_log2, m, l);
+                softmax_tile<HD, false>(tS, tO, tS + L::tP, j, BN, scale_log2, m, l, ctl.bar(L::bPHalf + i));
             else
-                softmax_tile<HD, true>(tS, tO, tS + L::tP, j, tail, scale_log2, m, l);
+                softmax_tile<HD, true>(tS, tO, tS + L::tP, j, tail, scale_log2, m, l, ctl.bar(L::bPHalf + i));
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(ctl.bar(L::bPFull + i));
