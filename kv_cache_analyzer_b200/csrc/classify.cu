@@ -17,7 +17,9 @@
 // buffered so one cluster barrier per pass suffices.  The tie pass counts
 // threshold ties per thread over a contiguous range, scans them inside the
 // CTA and across the 8 CTAs (again through distributed shared memory), then
-// writes the levels.  Exact and deterministic.
+// writes the levels.  Each CTA keeps its slice of keys in shared memory
+// (up to 40K keys, i.e. 320K scores per cluster; beyond that the passes
+// re-read them from L2).  Exact and deterministic.
 #include <cooperative_groups.h>
 
 #include "jano_common.cuh"
@@ -31,6 +33,7 @@ constexpr int kCluster = 8;
 constexpr int kThreads = 1024;
 constexpr int kBins = 2048;             // 11-bit digits
 constexpr int kPasses = 3;
+constexpr int kMaxCachedKeys = 40 * 1024;   // keys per CTA kept in shared memory (160 KB)
 __host__ __device__ constexpr int digit_shift(int pass) { return pass == 0 ? 21 : (pass == 1 ? 10 : 0); }
 __host__ __device__ constexpr int digit_width(int pass) { return pass == 2 ? 10 : 11; }
 
@@ -62,6 +65,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
 classify_kernel(const uint32_t* __restrict__ bits, int n, long long k_static,
                 long long k_active, uint8_t* __restrict__ levels, int* err) {
     __shared__ Shared sh;
+    extern __shared__ uint32_t cached[];     // this CTA's order keys, when they fit
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -73,11 +77,17 @@ classify_kernel(const uint32_t* __restrict__ bits, int n, long long k_static,
     const bool live0 = k_static > 0 && k_static < n;
     const bool live1 = k_active > 0 && k_active < n;
 
-    // ---- non-finite scores: any CTA seeing one makes the whole cluster stop
+    // ---- one coalesced sweep: non-finite check, keys into shared memory
+    const bool use_cache = hi - lo <= kMaxCachedKeys;
     int bad = 0;
-    for (int i = lo + tid; i < hi; i += kThreads)
-        bad |= (__ldg(bits + i) & 0x7F800000u) == 0x7F800000u;
+    for (int i = lo + tid; i < hi; i += kThreads) {
+        const uint32_t b = __ldg(bits + i);
+        bad |= (b & 0x7F800000u) == 0x7F800000u;
+        if (use_cache) cached[i - lo] = order_key(b);
+    }
     bad = __syncthreads_or(bad);
+    // key of element i (lo <= i < hi)
+    auto key = [&](int i) { return use_cache ? cached[i - lo] : order_key(__ldg(bits + i)); };
     if (tid == 0) {
         sh.bad = bad;
         sh.val[0] = sh.val[1] = 0u;
@@ -104,7 +114,7 @@ classify_kernel(const uint32_t* __restrict__ bits, int n, long long k_static,
         for (int base = lo; base < hi; base += kThreads) {
             const int i = base + tid;
             const bool ok = i < hi;
-            const uint32_t u = ok ? order_key(__ldg(bits + i)) : 0u;
+            const uint32_t u = ok ? key(i) : 0u;
             const unsigned dg = (u >> shift) & dmask;
             const bool m0 = ok && live0 && (u & hmask) == p0;
             const bool m1 = ok && live1 && (u & hmask) == p1;
@@ -155,7 +165,7 @@ classify_kernel(const uint32_t* __restrict__ bits, int n, long long k_static,
     const int tlo = min(hi, lo + tid * per_thr), thi = min(hi, tlo + per_thr);
     unsigned c0 = 0, c1 = 0;
     for (int i = tlo; i < thi; ++i) {
-        const uint32_t u = order_key(__ldg(bits + i));
+        const uint32_t u = key(i);
         c0 += live0 && u == v0;
         c1 += live1 && u == v1;
     }
@@ -184,7 +194,7 @@ classify_kernel(const uint32_t* __restrict__ bits, int n, long long k_static,
     }
     unsigned tie0 = b0 + w0 + s0 - c0, tie1 = b1 + w1 + s1 - c1;
     for (int i = tlo; i < thi; ++i) {
-        const uint32_t u = order_key(__ldg(bits + i));
+        const uint32_t u = key(i);
         const bool e0 = live0 && u == v0, e1 = live1 && u == v1;
         // rank < k_static ?  rank < k_active ?
         const bool below_s = live0 ? (u < v0 || (e0 && tie0 < need0)) : (k_static >= n);
@@ -201,8 +211,19 @@ classify_kernel(const uint32_t* __restrict__ bits, int n, long long k_static,
 cudaError_t launch_classify(const float* scores, int n, long long k_static,
                             long long k_active, uint8_t* levels, int* err,
                             cudaStream_t st) {
-    classify_kernel<<<kCluster, kThreads, 0, st>>>(reinterpret_cast<const uint32_t*>(scores), n,
-                                                   k_static, k_active, levels, err);
+    const int per_cta = (n + kCluster - 1) / kCluster;
+    const size_t smem = per_cta <= kMaxCachedKeys ? (size_t)per_cta * 4 : 0;
+    static unsigned long long done_mask = 0;   // per-device shared-memory opt-in
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !(done_mask & (1ull << dev))) {
+        cudaError_t e = cudaFuncSetAttribute(classify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kMaxCachedKeys * 4);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) done_mask |= 1ull << dev;
+    }
+    classify_kernel<<<kCluster, kThreads, smem, st>>>(reinterpret_cast<const uint32_t*>(scores), n,
+                                                      k_static, k_active, levels, err);
     return cudaGetLastError();
 }
 

@@ -12,8 +12,9 @@
 //              stored to scratch, per-level counts of the tile via warp ballots;
 //   2. scan    one CTA: per-level exclusive prefixes over tiles, per-step
 //              totals and the offsets[] prefix over steps;
-//   3. write   one CTA per (tile, step): ballot + popc prefix inside the tile,
-//              ascending stores of the due ids.
+//   3. write   one CTA per (tile, 8 steps): the tile's tokens ranked once in
+//              each of the four possible due sets (ballot + popc + one warp
+//              scan per set), then ascending stores of the due ids per step.
 // Scratch (caller-provided): token levels [n_tokens] u8, counts/prefixes
 // [3][n_tiles] int32 each.
 #include "jano_common.cuh"
@@ -140,27 +141,55 @@ scan_kernel(Ws ws, int n_tiles, jano_sched_cfg c, int32_t* __restrict__ offsets)
     }
 }
 
+// The due set of a step is one of four unions of levels: {3}, {3,2}, {3,1},
+// {3,2,1} (set id = due2 | due1 << 1).  Each CTA ranks its tile's tokens in
+// all four once (ballots + one warp scan per set) and then writes the lists
+// of kStepsPerCta consecutive steps from those ranks.
+constexpr int kStepsPerCta = 8;
+
 __global__ void __launch_bounds__(kTile)
 write_kernel(Ws ws, int n_tokens, int n_tiles, jano_sched_cfg c,
              const int32_t* __restrict__ offsets, int32_t* __restrict__ idx) {
-    __shared__ int wc[32];
+    __shared__ int wc[4][32];
+    __shared__ int wpre[4][32];
+    __shared__ int tpre[3];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int tile = blockIdx.x, s = blockIdx.y;
-    bool d2, d1;
-    step_due(s, c, d2, d1);
+    const int tile = blockIdx.x;
     const int t = tile * kTile + tid;
     const int lv = t < n_tokens ? ws.tok[t] : 0;
-    const bool due = t < n_tokens && level_due(lv, d2, d1);
-    const unsigned b = __ballot_sync(0xFFFFFFFFu, due);
-    if (lane == 0) wc[warp] = __popc(b);
+    const unsigned lt = (1u << lane) - 1u;
+    bool in[4];
+    int rank[4];
+#pragma unroll
+    for (int set = 0; set < 4; ++set) {
+        in[set] = t < n_tokens && level_due(lv, set & 1, (set >> 1) & 1);
+        const unsigned b = __ballot_sync(0xFFFFFFFFu, in[set]);
+        rank[set] = __popc(b & lt);
+        if (lane == 0) wc[set][warp] = __popc(b);
+    }
+    if (tid < 3) tpre[tid] = ws.pre[tid * n_tiles + tile];
     __syncthreads();
-    if (!due) return;
-    int wpre = 0;
-    for (int w = 0; w < warp; ++w) wpre += wc[w];
-    const long long base = (long long)offsets[s] + ws.pre[2 * n_tiles + tile] +
-                           (d2 ? ws.pre[1 * n_tiles + tile] : 0) +
-                           (d1 ? ws.pre[0 * n_tiles + tile] : 0);
-    idx[base + wpre + __popc(b & ((1u << lane) - 1u))] = t;
+    if (warp < 4) {
+        const int v = wc[warp][lane];
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        wpre[warp][lane] = incl - v;
+    }
+    __syncthreads();
+    const int s_end = min(c.T, (int)(blockIdx.y + 1) * kStepsPerCta);
+    for (int s = blockIdx.y * kStepsPerCta; s < s_end; ++s) {
+        bool d2, d1;
+        step_due(s, c, d2, d1);
+        const int set = (d2 ? 1 : 0) | (d1 ? 2 : 0);
+        if (in[set]) {
+            const long long base = (long long)offsets[s] + tpre[2] + (d2 ? tpre[1] : 0) + (d1 ? tpre[0] : 0);
+            idx[base + wpre[set][warp] + rank[set]] = t;
+        }
+    }
 }
 
 Geo make_geo(const jano_geom& g) {
@@ -193,7 +222,8 @@ cudaError_t launch_build_schedule(const uint8_t* block_levels, const jano_geom& 
     count_kernel<<<n_tiles, kTile, 0, st>>>(block_levels, geo, n_tokens, token_levels, ws,
                                              n_tiles, err);
     scan_kernel<<<1, kTile, 0, st>>>(ws, n_tiles, c, offsets);
-    write_kernel<<<dim3(n_tiles, c.T), kTile, 0, st>>>(ws, n_tokens, n_tiles, c, offsets, idx);
+    write_kernel<<<dim3(n_tiles, (c.T + kStepsPerCta - 1) / kStepsPerCta), kTile, 0, st>>>(
+        ws, n_tokens, n_tiles, c, offsets, idx);
     return cudaGetLastError();
 }
 

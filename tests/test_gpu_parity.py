@@ -116,7 +116,7 @@ def test_classify_gpu_scores_bit_exact_and_end_to_end(J, name):
     assert flips <= max(2, lv_gpu.size // 1000)
 
 
-@pytest.mark.parametrize("n", [1, 2, 7, 1023, 1024, 1025, 5000, 100_003])
+@pytest.mark.parametrize("n", [1, 2, 7, 1023, 1024, 1025, 5000, 100_003, 400_003])
 def test_classify_ties_and_sizes(J, n):
     g = np.random.default_rng(n)
     s = g.choice(np.array([-2.0, -0.0, 0.0, 0.5, 0.5, 1.0, 3.0], dtype=np.float32), size=n)
