@@ -33,7 +33,7 @@ import numpy as np
 __all__ = [
     "Workload", "WORKLOADS", "rng", "gaussian_blobs", "latent_history",
     "token_field", "bf16_bits", "bf16_normal", "bf16_perturb", "bf16_to_f32",
-    "normal_bf16", "perturb_bf16", "bits_of", "tensor_of",
+    "normal_bf16", "perturb_bf16", "bits_of", "tensor_of", "step_rows",
 ]
 
 
@@ -146,6 +146,13 @@ def tensor_of(bits: np.ndarray):
     """BF16 torch CPU tensor sharing memory with uint16 bit patterns."""
     import torch
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+
+def step_rows(tokens: np.ndarray, step: int, n_rows: int, shift: int = 7) -> np.ndarray:
+    """Pool rows that supply token ids `tokens` with fresh activations at
+    sampling step `step`: row (t + shift*step) mod n_rows.  A pure indexing
+    rule, so a few seeded pools stand in for new activations at every step."""
+    return (np.asarray(tokens, dtype=np.int64) + shift * step) % n_rows
 
 
 @dataclass(frozen=True)
