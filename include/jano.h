@@ -156,9 +156,9 @@ JANO_API jano_status jano_build_schedule(const uint8_t *block_levels, const jano
  * deployment convenience, not part of the method.
  *
  * Some callers cannot call cudaMalloc or any allocating routine where they
- * build the schedule (code running inside someone else's CUDA-graph
- * capture, runtimes without a device allocator, hosts whose memory pool
- * forbids side allocations).  This variant takes the same inputs and outputs
+ * build the schedule: plug-ins handed fixed buffers by a host framework,
+ * runtimes without a device allocator, hosts whose memory pool is owned by
+ * another framework and forbids side allocations.  This variant takes the same inputs and outputs
  * as jano_build_schedule but no workspace: its scratch is a file-scope
  * __device__ array of 1 MiB inside the library, which every GPU that loads
  * the library holds until the process exits.  It allocates nothing.

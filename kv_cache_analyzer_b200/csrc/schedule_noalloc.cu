@@ -2,9 +2,8 @@
 // for callers that cannot allocate device memory.
 //
 // Some callers cannot call cudaMalloc (or any allocating routine) at the
-// point where they build the schedule: code running while a CUDA graph is
-// being captured by someone else, allocator-less embedded runtimes, or hosts
-// whose memory pool is owned by another framework that forbids side
+// point where they build the schedule: plug-ins handed fixed buffers by a
+// host framework, allocator-less embedded runtimes, or hosts whose memory pool is owned by another framework that forbids side
 // allocations.  They still own the inputs and outputs; what they cannot
 // provide is the builder's scratch.  This entry point takes its scratch from
 // a fixed array in the library's own device image instead, so it allocates

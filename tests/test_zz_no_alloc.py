@@ -1,5 +1,5 @@
 """jano_build_schedule_noalloc, the schedule builder for callers that cannot
-allocate device memory (code inside someone else's CUDA-graph capture,
+allocate device memory (plug-ins handed fixed buffers by a host framework,
 runtimes without a device allocator, hosts whose pool forbids side
 allocations).  It uses the library's own 1 MiB device array as scratch
 instead of a caller workspace.
