@@ -56,8 +56,10 @@ def _load():
                                               i, i, i, i, i, P, P, ll, P]
         lib.oracle_kv_scatter.argtypes = [P, P, P, i, i, P, P, i]
         lib.oracle_active_attention.argtypes = [P, P, P, i, i, i, i, d, P, i, P]
+        lib.oracle_gather_gemm.argtypes = [P, i, P, i, P, i, i, P]
         for fn in ("oracle_block_scores", "oracle_level_counts", "oracle_classify",
-                   "oracle_build_schedule", "oracle_kv_scatter", "oracle_active_attention"):
+                   "oracle_build_schedule", "oracle_kv_scatter", "oracle_active_attention",
+                   "oracle_gather_gemm"):
             getattr(lib, fn).restype = C.c_int
         _lib = lib
     return _lib
@@ -144,4 +146,20 @@ def active_attention(q_act, k_cache, v_cache, scale=None, rows=None):
     _check("oracle_active_attention", _load().oracle_active_attention(
         _ptr(q), _ptr(kc), _ptr(vc), n_act, kc.shape[0], heads, d, float(scale),
         _ptr(rows), rows.shape[0], _ptr(out)))
+    return out
+
+
+def gather_gemm(x, w, gather=None):
+    """BF16 bits x [n_x][k], w [n][k], optional int32 gather [m] ->
+    fp64 [m][n] with out[r] = x[gather[r]] @ w^T (x[r] without gather)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    n_x, k = x.shape
+    n = w.shape[0]
+    assert w.shape[1] == k
+    g = None if gather is None else np.ascontiguousarray(gather, dtype=np.int32)
+    m = n_x if g is None else g.shape[0]
+    out = np.empty((m, n), dtype=np.float64)
+    _check("oracle_gather_gemm", _load().oracle_gather_gemm(
+        _ptr(x), n_x, _ptr(g), m, _ptr(w), n, k, _ptr(out)))
     return out

@@ -308,3 +308,37 @@ int oracle_active_attention(const uint16_t *q_act, const uint16_t *k_cache,
     free(s);
     return OR_OK;
 }
+
+/*
+ * Projections of the active tokens only (nl page, Methodologie 2 "KV Cache
+ * Mechanisme": per step JANO activates only a subset of the tokens and
+ * stores the K/V of the frozen ones, so the DiT block's linear maps run on
+ * the active rows alone; zh page 2.2 item 3).  A linear map y = x W^T on the
+ * rows of x picked by `gather` (row r reads x[gather[r]]; gather == NULL
+ * reads x[r]):
+ *
+ *   out[r][j] = sum_c x[src(r)][c] * w[j][c],   r < m, j < n
+ *
+ * x is [n_x][k] and w [n][k] BF16 bit patterns (w in the usual [out][in]
+ * layout of a linear layer), decoded exactly; the sums are fp64 in c order.
+ * out is [m][n] fp64.  Where the rows land (a token-ordered buffer, the K/V
+ * cache) is placement only and is checked separately by the tests.
+ */
+int oracle_gather_gemm(const uint16_t *x, int n_x, const int32_t *gather, int m,
+                       const uint16_t *w, int n, int k, double *out)
+{
+    if (!x || !w || !out || n_x < 1 || m < 0 || n < 1 || k < 1) return OR_EINVAL;
+    for (int r = 0; r < m; ++r) {
+        const int src = gather ? gather[r] : r;
+        if (src < 0 || src >= n_x) return OR_EINDEX;
+        const uint16_t *xr = x + (size_t)src * k;
+        for (int j = 0; j < n; ++j) {
+            const uint16_t *wj = w + (size_t)j * k;
+            double acc = 0.0;
+            for (int c = 0; c < k; ++c)
+                acc += bf16_value(xr[c]) * bf16_value(wj[c]);
+            out[(size_t)r * n + j] = acc;
+        }
+    }
+    return OR_OK;
+}

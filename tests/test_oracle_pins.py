@@ -409,3 +409,71 @@ def test_bf16_rounding_matches_torch():
     ours = synth.bf16_bits(x)
     ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     np.testing.assert_array_equal(ours, ref)
+
+
+# ---------------------------------------------------------------- projections of the active rows
+def _bits(a):
+    return synth.bf16_bits(np.asarray(a, dtype=np.float32))
+
+
+def test_gather_gemm_hand_example():
+    g = golden("gather_gemm_hand.json")
+    got = oracle.gather_gemm(_bits(g["x"]), _bits(g["w"]), np.array(g["gather"], dtype=np.int32))
+    np.testing.assert_array_equal(got, np.array(g["expected"]))
+
+
+def test_gather_gemm_identity_weight_gathers_rows_exactly():
+    gen = np.random.default_rng(31)
+    x = synth.bf16_normal((40, 24), gen)
+    gather = gen.integers(0, 40, size=17).astype(np.int32)
+    eye = _bits(np.eye(24))
+    got = oracle.gather_gemm(x, eye, gather)
+    np.testing.assert_array_equal(got, synth.bf16_to_f32(x)[gather].astype(np.float64))
+
+
+def test_gather_gemm_matches_library_matmul():
+    # the same product by numpy's fp64 matmul and by torch's fp64 linear layer
+    import torch
+    gen = np.random.default_rng(32)
+    x, w = synth.bf16_normal((50, 72), gen), synth.bf16_normal((30, 72), gen)
+    gather = gen.integers(0, 50, size=23).astype(np.int32)
+    got = oracle.gather_gemm(x, w, gather)
+    xf, wf = synth.bf16_to_f32(x).astype(np.float64), synth.bf16_to_f32(w).astype(np.float64)
+    np.testing.assert_allclose(got, xf[gather] @ wf.T, rtol=1e-12, atol=1e-12)
+    tl = torch.nn.functional.linear(torch.from_numpy(xf[gather]), torch.from_numpy(wf)).numpy()
+    np.testing.assert_allclose(got, tl, rtol=1e-12, atol=1e-12)
+
+
+def test_gather_gemm_rows_follow_the_gather_and_default_to_identity():
+    gen = np.random.default_rng(33)
+    x, w = synth.bf16_normal((12, 16), gen), synth.bf16_normal((8, 16), gen)
+    full = oracle.gather_gemm(x, w)                       # no gather: row r reads x[r]
+    perm = gen.permutation(12).astype(np.int32)
+    np.testing.assert_array_equal(oracle.gather_gemm(x, w, perm), full[perm])
+    np.testing.assert_array_equal(oracle.gather_gemm(x, w, np.array([5, 5], dtype=np.int32)), full[[5, 5]])
+
+
+def test_gather_gemm_is_linear_in_the_weight_and_transposes_right():
+    # a wrong operand orientation (x @ w instead of x @ w^T) or a dropped
+    # term breaks these: one-hot weight rows pick single input columns
+    gen = np.random.default_rng(34)
+    x = synth.bf16_normal((9, 6), gen)
+    onehot = np.zeros((3, 6), dtype=np.float32)
+    onehot[0, 5] = 1.0
+    onehot[1, 0] = 1.0
+    onehot[2, 2] = -2.0
+    got = oracle.gather_gemm(x, _bits(onehot))
+    xf = synth.bf16_to_f32(x).astype(np.float64)
+    np.testing.assert_array_equal(got[:, 0], xf[:, 5])
+    np.testing.assert_array_equal(got[:, 1], xf[:, 0])
+    np.testing.assert_array_equal(got[:, 2], -2.0 * xf[:, 2])
+    w1, w2 = synth.bf16_normal((4, 6), gen), synth.bf16_normal((4, 6), gen)
+    both = np.concatenate([w1, w2])
+    np.testing.assert_array_equal(oracle.gather_gemm(x, both),
+                                  np.concatenate([oracle.gather_gemm(x, w1), oracle.gather_gemm(x, w2)], axis=1))
+
+
+def test_gather_gemm_rejects_out_of_range_row():
+    x = _bits(np.ones((4, 8)))
+    with pytest.raises(oracle.OracleError):
+        oracle.gather_gemm(x, x, np.array([0, 4], dtype=np.int32))
