@@ -226,6 +226,57 @@ JANO_API jano_status jano_active_attention(const void *q_act, const void *k_cach
                                   int n_act, int n_tokens, int heads, int d,
                                   float scale, void *out, void *stream);
 
+/* ------------------------------------------------------------------------
+ * jano_gather_gemm -- a linear layer on the active rows only, rows gathered
+ * on the way in and optionally scattered on the way out.  Pages: nl
+ * technical summary, Methodologie 2 "KV Cache Mechanisme" (per step only a
+ * subset of the tokens is activated; the K/V of the frozen ones are kept),
+ * so the DiT block's projections run on the active rows alone; zh 2.2
+ * item 3.
+ *
+ *   for r < m:  out[dst(r)][j] = sum_c x[src(r)][c] * w[j][c]
+ *   src(r) = gather ? gather[r] : r,   dst(r) = scatter ? scatter[r] : r
+ *
+ * x        device BF16 [n_x][k] (e.g. the hidden states of all tokens).
+ * gather   device int32 [m] or NULL; values in [0, n_x).  Without it m <= n_x.
+ * w        device BF16 [n][k]: a linear layer's weight in [out][in] layout.
+ * scatter  device int32 [m] or NULL; values in [0, n_out).  Without it
+ *          m <= n_out.  Two active rows must not share a destination.
+ * out      device BF16 [n_out][n]; rows not written keep their contents.
+ * k % 8 == 0 and n % 8 == 0 (JANO_EUNSUPPORTED otherwise); x, w, out
+ * 16-byte aligned.  BF16 in, fp32 accumulation on the tensor cores, BF16
+ * out (round to nearest even).  An index out of range raises JANO_EINDEX on
+ * the device error word: a bad gather index reads a row of zeros, a bad
+ * scatter index drops the row.  m == 0 is a no-op.
+ * ---------------------------------------------------------------------- */
+JANO_API jano_status jano_gather_gemm(const void *x, int n_x, const int32_t *gather, int m,
+                                      const void *w, int n, int k, const int32_t *scatter,
+                                      void *out, int n_out, void *stream);
+
+/* ------------------------------------------------------------------------
+ * jano_qkv_project -- the fused Q/K/V projection of the active tokens with
+ * the KV-cache write (same passages as jano_gather_gemm, plus the KV cache
+ * of Methodologie 2): with y_i = x[idx[i]] @ w_qkv^T,
+ *
+ *   q_act[i]        = y_i[0 .. hd)
+ *   k_cache[idx[i]] = y_i[hd .. 2hd)
+ *   v_cache[idx[i]] = y_i[2hd .. 3hd)
+ *
+ * so the fresh K/V rows go straight from the tensor cores into the
+ * token-ordered cache: no K_act/V_act buffers and no separate
+ * jano_kv_scatter.  hd = heads * d.
+ *
+ * x        device BF16 [n_tokens][k], the hidden states of all tokens.
+ * idx      device int32 [n_act], the active tokens (distinct, in [0, n_tokens)).
+ * w_qkv    device BF16 [3*hd][k]: the Q rows, then the K rows, then the V rows.
+ * q_act    device BF16 [n_act][hd]; k_cache, v_cache device BF16 [n_tokens][hd].
+ * hd must be a multiple of 128 and k of 8 (JANO_EUNSUPPORTED otherwise);
+ * pointers 16-byte aligned.  Errors as for jano_gather_gemm.
+ * ---------------------------------------------------------------------- */
+JANO_API jano_status jano_qkv_project(const void *x, int n_tokens, const int32_t *idx, int n_act,
+                                      const void *w_qkv, int hd, int k, void *q_act,
+                                      void *k_cache, void *v_cache, void *stream);
+
 /* Synchronises `stream`, returns the first device-side error recorded on the
  * current device since the last call (JANO_OK if none) and clears it. */
 JANO_API jano_status jano_get_device_error(void *stream);

@@ -38,6 +38,7 @@ STATUS_NAMES = {0: "JANO_OK", 1: "JANO_EINVAL", 2: "JANO_ESHAPE", 3: "JANO_EALIG
                 7: "JANO_ETIMEOUT", 8: "JANO_ECUDA"}
 EXPORTS = ("jano_block_scores", "jano_classify", "jano_build_schedule_workspace_bytes",
            "jano_build_schedule", "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention",
+           "jano_gather_gemm", "jano_qkv_project",
            "jano_get_device_error", "jano_status_str", "jano_version")
 
 
@@ -76,13 +77,15 @@ def lib() -> C.CDLL:
         L.jano_build_schedule_noalloc.argtypes = [P, G, S, P, P, z, P, P]
         L.jano_kv_scatter.argtypes = [P, P, P, i, i, i, P, P, i, P]
         L.jano_active_attention.argtypes = [P, P, P, P, i, i, i, i, f, P, P]
+        L.jano_gather_gemm.argtypes = [P, i, P, i, P, i, i, P, P, i, P]
+        L.jano_qkv_project.argtypes = [P, i, P, i, P, i, i, P, P, P, P]
         L.jano_get_device_error.argtypes = [P]
         L.jano_status_str.argtypes = [i]
         L.jano_status_str.restype = C.c_char_p
         L.jano_version.argtypes = []
         for fn in ("jano_block_scores", "jano_classify", "jano_build_schedule",
                    "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention", "jano_get_device_error",
-                   "jano_version"):
+                   "jano_gather_gemm", "jano_qkv_project", "jano_version"):
             getattr(L, fn).restype = C.c_int
         _lib = L
     return _lib
@@ -164,6 +167,21 @@ def jano_active_attention(q_act, k_cache, v_cache, idx, n_act, n_tokens, heads, 
         _dev(q_act, "q_act", torch.bfloat16), _dev(k_cache, "k_cache", torch.bfloat16),
         _dev(v_cache, "v_cache", torch.bfloat16), _dev(idx, "idx", torch.int32), n_act,
         n_tokens, heads, d, scale, _dev(out, "out", torch.bfloat16), _stream(stream)))
+
+
+def jano_gather_gemm(x, n_x, gather, m, w, n, k, scatter, out, n_out, stream=None):
+    _check("jano_gather_gemm", lib().jano_gather_gemm(
+        _dev(x, "x", torch.bfloat16), n_x, _dev(gather, "gather", torch.int32), m,
+        _dev(w, "w", torch.bfloat16), n, k, _dev(scatter, "scatter", torch.int32),
+        _dev(out, "out", torch.bfloat16), n_out, _stream(stream)))
+
+
+def jano_qkv_project(x, n_tokens, idx, n_act, w_qkv, hd, k, q_act, k_cache, v_cache, stream=None):
+    _check("jano_qkv_project", lib().jano_qkv_project(
+        _dev(x, "x", torch.bfloat16), n_tokens, _dev(idx, "idx", torch.int32), n_act,
+        _dev(w_qkv, "w_qkv", torch.bfloat16), hd, k, _dev(q_act, "q_act", torch.bfloat16),
+        _dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
+        _stream(stream)))
 
 
 def jano_get_device_error(stream=None) -> int:
@@ -261,6 +279,24 @@ def active_attention(q_act, k_cache, v_cache, idx, out, scale=None, stream=None)
     if scale is None:
         scale = d ** -0.5
     jano_active_attention(q_act, k_cache, v_cache, idx, n_act, N, H, d, scale, out, stream)
+
+
+def gather_gemm(x, w, out, gather=None, scatter=None, stream=None) -> None:
+    """out[scatter[r] or r] = x[gather[r] or r] @ w^T for r < m (BF16 tensors
+    x [n_x][k], w [n][k], out [n_out][n]; m = len(gather or scatter or x))."""
+    n_x, k = x.shape
+    n = w.shape[0]
+    m = gather.numel() if gather is not None else (scatter.numel() if scatter is not None else n_x)
+    jano_gather_gemm(x, n_x, gather, m, w, n, k, scatter, out, out.shape[0], stream)
+
+
+def qkv_project(x, idx, w_qkv, q_act, k_cache, v_cache, stream=None) -> None:
+    """Q/K/V of the active tokens idx from the hidden states x [N][k]:
+    q_act [n_act][hd] and the rows idx of k_cache, v_cache [N][hd] (also
+    accepted as [N][heads][d])."""
+    N, k = x.shape
+    hd = w_qkv.shape[0] // 3
+    jano_qkv_project(x, N, idx, idx.numel(), w_qkv, hd, k, q_act, k_cache, v_cache, stream)
 
 
 def device_error(stream=None) -> int:

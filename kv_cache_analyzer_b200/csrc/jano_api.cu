@@ -146,6 +146,42 @@ jano_status jano_active_attention(const void* q_act, const void* k_cache, const 
                                              d, scale, out, err, static_cast<cudaStream_t>(stream)));
 }
 
+jano_status jano_gather_gemm(const void* x, int n_x, const int32_t* gather, int m, const void* w,
+                             int n, int k, const int32_t* scatter, void* out, int n_out,
+                             void* stream) {
+    if (n_x < 1 || m < 0 || n < 1 || k < 1 || n_out < 1) return JANO_EINVAL;
+    if (m == 0) return JANO_OK;
+    if (!x || !w || !out) return JANO_EINVAL;
+    if (!gather && m > n_x) return JANO_ESHAPE;
+    if (!scatter && m > n_out) return JANO_ESHAPE;
+    if (k % 8 || n % 8) return JANO_EUNSUPPORTED;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(out)) return JANO_EALIGN;
+    int* err = device_error_word();
+    if (!err) return JANO_ECUDA;
+    ProjSeg seg{out, scatter, n, n_out};
+    return from_cuda(launch_projection(x, n_x, gather, m, w, n, k, 1, &seg, err,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+jano_status jano_qkv_project(const void* x, int n_tokens, const int32_t* idx, int n_act,
+                             const void* w_qkv, int hd, int k, void* q_act, void* k_cache,
+                             void* v_cache, void* stream) {
+    if (n_tokens < 1 || n_act < 0 || hd < 1 || k < 1) return JANO_EINVAL;
+    if (n_act == 0) return JANO_OK;
+    if (!x || !idx || !w_qkv || !q_act || !k_cache || !v_cache) return JANO_EINVAL;
+    if (k % 8 || projection_tile_n(3 * hd, hd, 3) == 0) return JANO_EUNSUPPORTED;
+    if (3ll * hd > INT_MAX) return JANO_EUNSUPPORTED;
+    if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(q_act) || !aligned16(k_cache) ||
+        !aligned16(v_cache))
+        return JANO_EALIGN;
+    int* err = device_error_word();
+    if (!err) return JANO_ECUDA;
+    const ProjSeg segs[3] = {{q_act, nullptr, hd, n_act}, {k_cache, idx, hd, n_tokens},
+                             {v_cache, idx, hd, n_tokens}};
+    return from_cuda(launch_projection(x, n_tokens, idx, n_act, w_qkv, 3 * hd, k, 3, segs, err,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 jano_status jano_get_device_error(void* stream) {
     int* err = device_error_word();
     if (!err) return JANO_ECUDA;

@@ -45,6 +45,21 @@ cudaError_t launch_active_attention(const void* q, const void* k, const void* v,
                                     int heads, int d, float scale, void* out,
                                     int* err, cudaStream_t st);
 
+// One output segment of the projection kernel: its columns go to `dst`
+// (BF16 rows of `ld` elements) at row rowmap[r] (or r when rowmap is NULL).
+struct ProjSeg {
+    void* dst;
+    const int32_t* rowmap;
+    int ld;
+    int n_rows;
+};
+// y = x[gather] w^T on m rows; the n columns are cut into n_seg equal
+// segments (1..3), each stored through its ProjSeg.
+cudaError_t launch_projection(const void* x, int n_x, const int32_t* gather, int m, const void* w,
+                              int n, int k, int n_seg, const ProjSeg* segs, int* err,
+                              cudaStream_t st);
+int projection_tile_n(int n, int seg_w, int n_seg);
+
 namespace ptx {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -123,6 +123,15 @@ def normal_bf16(shape, seed):
     return torch.randn(tuple(shape), generator=g, dtype=torch.float32).to(torch.bfloat16)
 
 
+def linear_weight_bf16(n_out, n_in, seed):
+    """Random linear-layer weight [n_out][n_in]: N(0, 1/n_in) rounded to BF16
+    (torch CPU tensor, seeded), so x @ w^T keeps unit-scale activations."""
+    import torch
+    g = torch.Generator().manual_seed(int(seed))
+    w = torch.randn((n_out, n_in), generator=g, dtype=torch.float32) * (n_in ** -0.5)
+    return w.to(torch.bfloat16)
+
+
 def perturb_bf16(x, sigma, seed):
     """BF16(x + N(0, sigma^2)) for a BF16 torch CPU tensor x (a stale cache)."""
     import torch

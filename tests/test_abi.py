@@ -84,6 +84,15 @@ def test_host_validation_rejects_before_any_launch(jl):
     ok = jl.Schedule(T=4, warmup=1, cooldown=1).c()
     assert L.jano_build_schedule(fake, C.byref(g3), C.byref(ok), fake, fake, 10, nil, fake,
                                  10**6, nil) == 1
+    # projections: k or n not a multiple of 8, misaligned operand, m beyond
+    # the rows without a gather, an empty call, hd not a multiple of 128
+    assert L.jano_gather_gemm(fake, 64, nil, 16, fake, 60, 64, nil, fake, 64, nil) == 4
+    assert L.jano_gather_gemm(fake, 64, nil, 16, fake, 64, 60, nil, fake, 64, nil) == 4
+    assert L.jano_gather_gemm(C.c_void_p(264), 64, nil, 16, fake, 64, 64, nil, fake, 64, nil) == 3
+    assert L.jano_gather_gemm(fake, 8, nil, 16, fake, 64, 64, nil, fake, 64, nil) == 2
+    assert L.jano_gather_gemm(nil, 8, nil, 0, nil, 64, 64, nil, nil, 64, nil) == 0
+    assert L.jano_qkv_project(fake, 100, fake, 10, fake, 96, 64, fake, fake, fake, nil) == 4
+    assert L.jano_qkv_project(nil, 100, nil, 0, nil, 128, 64, nil, nil, nil, nil) == 0
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch, jl):
