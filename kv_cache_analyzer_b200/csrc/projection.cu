@@ -15,9 +15,10 @@
 //            straight into the 128-byte-swizzled K-major layout the tensor
 //            core reads (chunk c of row i at i*128 + ((c ^ (i % 8)) * 16));
 //            the weight rows come by one tiled TMA box.  A 4-slot ring; each
-//            producer thread keeps up to three stages of copies in flight and
-//            signals a stage once its copies have landed (cp.async.wait_group,
-//            then a generic-to-async proxy fence, then an mbarrier arrive).
+//            producer thread hands a stage over with cp.async.mbarrier.arrive
+//            (the barrier cannot complete before that thread's copies have
+//            landed) plus an ordinary arrive, so it never waits for its own
+//            copies and runs as far ahead as the ring allows.
 //   warp 4   allocates BN TMEM columns; one lane issues tcgen05.mma
 //            (kind::f16, M=128, N=BN, K=16, both operands K-major from shared
 //            memory, fp32 accumulator in TMEM) and frees ring slots with
@@ -49,7 +50,6 @@ constexpr int kStages = 4;
 constexpr int kProducers = 128;         // warps 0-3
 constexpr int kMmaWarp = 4;
 constexpr int kThreads = 288;
-constexpr int kLag = kStages - 1;       // stages a producer keeps in flight
 constexpr int kGroupM = 16;             // row tiles per rasterisation group
 constexpr long long kWaitLimit = 1ll << 31;
 
@@ -112,11 +112,14 @@ struct PCtl {
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-// Make this thread's completed generic-proxy writes to shared memory visible
-// to the async proxy (the tensor core reads its operands through it).
+// Arrive on `bar` once every cp.async this thread issued so far has landed
+// (the barrier's pending count is raised first, so the phase waits for it).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Order shared-memory writes this thread has observed (through an mbarrier)
+// before its following async-proxy accesses (the tensor core's operand reads).
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1) {
@@ -202,15 +205,14 @@ projection_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
         int src[PM / 16];
 #pragma unroll
         for (int u = 0; u < PM / 16; ++u) src[u] = rows[rg + 16 * u];
-        int kb = 0, signalled = 0;
-        bool ok = true;
+        int kb = 0;
         for (; kb < nkb; ++kb) {
             const int s = kb % kStages;
             // warp-uniform: lane 0 waits, the warp follows
-            if (!ctl.warp_wait(L::bEmpty + s, ((kb / kStages) & 1) ^ 1)) { ok = false; break; }
+            if (!ctl.warp_wait(L::bEmpty + s, ((kb / kStages) & 1) ^ 1)) break;
             const uint32_t sa = base + s * L::kStage;
+            const uint32_t full = ctl.bar(L::bFull + s);
             if (t == 0) {
-                const uint32_t full = ctl.bar(L::bFull + s);
                 ptx::mbar_arrive_expect_tx(full, L::kB);
                 tma_load_2d(sa + L::kA, &tmB, full, kb * PK, n0);
             }
@@ -223,20 +225,11 @@ projection_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
                 const void* g = live ? static_cast<const void*>(xb + (size_t)src[u] * a.k + col) : a.x;
                 cp_async16(sa + i * 128 + ((c ^ (i & 7)) << 4), g, live ? 16u : 0u);
             }
-            cp_async_commit();
-            if (kb >= kLag) {
-                // stage kb - kLag has landed: publish it to the tensor core
-                cp_async_wait<kLag>();
-                fence_proxy_async();
-                ptx::mbar_arrive(ctl.bar(L::bFull + (kb - kLag) % kStages));
-                ++signalled;
-            }
+            cp_async_arrive(full);
+            ptx::mbar_arrive(full);
         }
-        // the last stages (all of them after a timeout, so no copy outlives the CTA)
-        cp_async_wait<0>();
-        fence_proxy_async();
-        if (ok)
-            for (int q = signalled; q < nkb; ++q) ptx::mbar_arrive(ctl.bar(L::bFull + q % kStages));
+        // no copy outlives the CTA (after a timeout some stages are never consumed)
+        cp_async_wait_all();
         if (t == 0) {
             // drain: every weight copy this CTA issued lands before its smem is released
             for (int q = (kb > kStages ? kb - kStages : 0); q < kb; ++q)
@@ -250,6 +243,7 @@ projection_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
             for (int kb = 0; kb < nkb; ++kb) {
                 const int s = kb % kStages;
                 if (!ctl.wait(L::bFull + s, (kb / kStages) & 1)) { ok = false; break; }
+                fence_proxy_async();
                 ptx::tc_fence_after();
                 const uint32_t sa = base + s * L::kStage;
 #pragma unroll
