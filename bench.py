@@ -1,7 +1,7 @@
 """Benchmark of the Jano hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload large]
-                    [--impl reference] [--no-cpu-baseline] [--no-e2e]
+                    [--impl reference] [--no-cpu-baseline] [--no-e2e] [--no-next]
 
 One step = one pass of the whole hot path over one batch of synthetic input
 (block scores over the latent history, level split of the per-token field,
@@ -13,6 +13,11 @@ divided by the whole step's device time (max over ranks); the analyzer and
 scatter HBM GB/s and per-kernel times are reported beside it.  Every rank
 runs an independent replica of the workload (a different seed): the path
 has no data-path exchange, so N GPUs process N problems ("weak" scaling).
+
+Beside the step (not in its value) the line reports ``next_rows``: the
+block's projections on the step's active tokens -- the fused Q/K/V projection
+writing K/V straight into the cache and the output projection scattered back
+to the token rows -- with their TFLOP/s.
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead, on
 a bounded sample of the same workload, extrapolated stage by stage to the
@@ -205,6 +210,49 @@ def cpu_oracle_step_time(w, inp, k_cache, v_cache, budget_rows=8, rng_seed=0):
     return est, flops, "; ".join(parts) + " (single-threaded fp64 C, extrapolated per stage)"
 
 
+def measure_projections(J, hp, step, stream, pk, reps=10):
+    """The block's projections on the step's active tokens (outside the hot
+    path's step, reported beside it): the fused Q/K/V projection that writes
+    K/V straight into the cache, and the output projection scattered back to
+    the token rows.  Random-init weights N(0, 1/k) in BF16; hidden states
+    N(0, 1) for every token (hidden size heads x d)."""
+    import torch
+    start, n_act = hp.due(step)
+    idx = hp.idx[start:start + n_act]
+    N, hd = hp.N, hp.heads * hp.d
+    g = torch.Generator(device=hp.dev).manual_seed(1234)
+    x = torch.randn((N, hd), generator=g, device=hp.dev).to(torch.bfloat16)
+    w_qkv = (torch.randn((3 * hd, hd), generator=g, device=hp.dev) * hd ** -0.5).to(torch.bfloat16)
+    w_o = (torch.randn((hd, hd), generator=g, device=hp.dev) * hd ** -0.5).to(torch.bfloat16)
+    q = torch.empty((n_act, hd), dtype=torch.bfloat16, device=hp.dev)
+    o_act = torch.randn((n_act, hd), generator=g, device=hp.dev).to(torch.bfloat16)
+    y = torch.zeros((N, hd), dtype=torch.bfloat16, device=hp.dev)
+    kc, vc = hp.k_cache.view(N, hd), hp.v_cache.view(N, hd)
+    ops = {
+        "qkv_project": (lambda: J.qkv_project(x, idx, w_qkv, q, kc, vc, stream), 2.0 * n_act * 3 * hd * hd),
+        "out_proj_scatter": (lambda: J.gather_gemm(o_act, w_o, y, scatter=idx, stream=stream),
+                             2.0 * n_act * hd * hd),
+    }
+    res = {}
+    for name, (fn, flops) in ops.items():
+        for _ in range(3):
+            fn()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        evs[0].record(stream)
+        for i in range(reps):
+            fn()
+            evs[i + 1].record(stream)
+        stream.synchronize()
+        ms = sorted(evs[i].elapsed_time(evs[i + 1]) for i in range(reps))[reps // 2]
+        tf = flops / (ms * 1e-3) / 1e12
+        res[name] = {"ms": ms, "TFLOP/s": tf, "flops": flops, "frac_of_burst_peak": tf / pk["bf16_tflops"],
+                     "shape": {"m": n_act, "n": (3 if name == "qkv_project" else 1) * hd, "k": hd}}
+    code = J.device_error(stream)
+    if code:
+        raise RuntimeError(f"device error in projections: {J.jano_status_str(code)}")
+    return res
+
+
 def run_reference(args, w, rank, world):
     if rank != 0:
         return 0
@@ -356,6 +404,10 @@ def run_gpu(args, w, rank, world, local_rank, dist):
         cpu = {"value": fl / est / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
                "sample": sample, "wall_s": time.perf_counter() - t0}
 
+    next_rows = None
+    if not args.no_next:
+        next_rows = measure_projections(J, hp, step, stream, pk)
+
     cfg = workload_config(w)
     cfg.update({"n_active": n_act, "global_batch": world, "parallelism": f"replicas x{world}",
                 "l2": "no flush: the per-step working set (K/V cache 1.5 GB, Q/K/V act 0.6 GB) "
@@ -365,7 +417,8 @@ def run_gpu(args, w, rank, world, local_rank, dist):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": cfg, "roofline": roofline, "cpu_baseline": cpu,
             "e2e": e2e, "gpu_launches": KERNELS_PER_STEP * args.steps, "clocks": clk.summary(),
-            "kernels": kernels, "peaks": {"source": pk_src, "hbm_gbs": hbm,
+            "kernels": kernels, "next_rows": next_rows,
+            "peaks": {"source": pk_src, "hbm_gbs": hbm,
                                           "bf16_tflops": pk["bf16_tflops"],
                                           "bf16_tflops_sustained": bf16_sus}}
     print(json.dumps(line), flush=True)
@@ -382,6 +435,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=8)
+    ap.add_argument("--no-next", action="store_true",
+                    help="skip the projections measured beside the step")
     args = ap.parse_args()
 
     import synth
