@@ -57,9 +57,12 @@ def _load():
         lib.oracle_kv_scatter.argtypes = [P, P, P, i, i, P, P, i]
         lib.oracle_active_attention.argtypes = [P, P, P, i, i, i, i, d, P, i, P]
         lib.oracle_gather_gemm.argtypes = [P, i, P, i, P, i, i, P]
+        lib.oracle_splitmix64.argtypes = [C.c_uint64, i, P]
+        lib.oracle_splitmix64.restype = None
+        lib.oracle_random_scores.argtypes = [i, C.c_uint64, P]
         for fn in ("oracle_block_scores", "oracle_level_counts", "oracle_classify",
                    "oracle_build_schedule", "oracle_kv_scatter", "oracle_active_attention",
-                   "oracle_gather_gemm"):
+                   "oracle_gather_gemm", "oracle_random_scores"):
             getattr(lib, fn).restype = C.c_int
         _lib = lib
     return _lib
@@ -162,4 +165,18 @@ def gather_gemm(x, w, gather=None):
     out = np.empty((m, n), dtype=np.float64)
     _check("oracle_gather_gemm", _load().oracle_gather_gemm(
         _ptr(x), n_x, _ptr(g), m, _ptr(w), n, k, _ptr(out)))
+    return out
+
+
+def splitmix64(seed, n):
+    """The first n outputs of splitmix64 seeded with `seed` (uint64)."""
+    out = np.empty(n, dtype=np.uint64)
+    _load().oracle_splitmix64(C.c_uint64(seed), n, _ptr(out))
+    return out
+
+
+def random_scores(n, seed):
+    """Uniform [0, 1) fp32 scores of the random-masking ablation (24 bits)."""
+    out = np.empty(n, dtype=np.float32)
+    _check("oracle_random_scores", _load().oracle_random_scores(n, C.c_uint64(seed), _ptr(out)))
     return out

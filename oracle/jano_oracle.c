@@ -342,3 +342,43 @@ int oracle_gather_gemm(const uint16_t *x, int n_x, const int32_t *gather, int m,
     }
     return OR_OK;
 }
+
+/*
+ * Random-masking ablation (ko page, section 4 "Ablation Study": random
+ * masking at a similar speed-up gives clearly worse quality than Jano's
+ * convergence-aware levels).  The ablation keeps Jano's level counts but
+ * assigns the levels at random: block b gets the uniform score
+ *
+ *   u_b = (splitmix64 output number b+1 of the stream seeded with `seed`) >> 40, times 2^-24
+ *
+ * and the scores are classified exactly like the analyzer's (same counts,
+ * ties by block index).  splitmix64 (Steele, Lea and Flood, "Fast splittable
+ * pseudorandom number generators", 2014): the state advances by the golden
+ * gamma 0x9E3779B97F4A7C15 and each output is the state passed through the
+ * 64-bit finaliser (xor-shift 30, multiply 0xBF58476D1CE4E5B9, xor-shift 27,
+ * multiply 0x94D049BB133111EB, xor-shift 31).  Output number i (from 1) is
+ * therefore a function of seed + i * gamma alone.
+ */
+void oracle_splitmix64(uint64_t seed, int n, uint64_t *out)
+{
+    uint64_t state = seed;
+    for (int i = 0; i < n; ++i) {
+        state += 0x9E3779B97F4A7C15ull;
+        uint64_t z = state;
+        z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+        z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+        out[i] = z ^ (z >> 31);
+    }
+}
+
+int oracle_random_scores(int n, uint64_t seed, float *scores)
+{
+    if (n < 1 || !scores) return OR_EINVAL;
+    uint64_t *r = (uint64_t *)malloc((size_t)n * sizeof(uint64_t));
+    if (!r) return OR_ENOMEM;
+    oracle_splitmix64(seed, n, r);
+    for (int b = 0; b < n; ++b)
+        scores[b] = (float)((double)(r[b] >> 40) / 16777216.0);   /* exact: 24-bit integer / 2^24 */
+    free(r);
+    return OR_OK;
+}

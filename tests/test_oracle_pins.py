@@ -477,3 +477,35 @@ def test_gather_gemm_rejects_out_of_range_row():
     x = _bits(np.ones((4, 8)))
     with pytest.raises(oracle.OracleError):
         oracle.gather_gemm(x, x, np.array([0, 4], dtype=np.int32))
+
+
+# ---------------------------------------------------------------- random-masking ablation
+def test_splitmix64_known_answers():
+    g = golden("splitmix64_seed0.json")
+    got = oracle.splitmix64(g["seed"], 4)
+    assert [f"{int(v):016x}" for v in got] == g["expected_hex"]
+
+
+def test_random_scores_follow_the_stream_and_are_uniform():
+    n, seed = 200000, 12345
+    s = oracle.random_scores(n, seed)
+    raw = oracle.splitmix64(seed, n)
+    # the score is the top 24 bits of output b+1, exactly
+    np.testing.assert_array_equal(s, ((raw >> np.uint64(40)).astype(np.float64) / 2**24).astype(np.float32))
+    assert s.min() >= 0.0 and s.max() < 1.0
+    # uniform: mean, variance and a 20-bin chi-square (df 19; 60 is far past p = 1e-6)
+    assert abs(s.mean() - 0.5) < 5 / math.sqrt(12 * n)
+    assert abs(s.var() - 1 / 12) < 0.002
+    hist = np.histogram(s, bins=20, range=(0, 1))[0]
+    chi2 = ((hist - n / 20) ** 2 / (n / 20)).sum()
+    assert chi2 < 60
+    # another seed gives another stream
+    assert not np.array_equal(s[:100], oracle.random_scores(100, seed + 1))
+
+
+def test_random_level_map_keeps_the_level_counts():
+    # the ablation assigns Jano's level counts at random: same n_A / n_S
+    n = 19320
+    lv = oracle.classify(oracle.random_scores(n, 7), 0.25, 0.45)
+    n_a, n_s = oracle.level_counts(n, 0.25, 0.45)
+    assert (lv == 3).sum() == n_a and (lv == 1).sum() == n_s and (lv == 2).sum() == n - n_a - n_s
