@@ -277,6 +277,24 @@ JANO_API jano_status jano_qkv_project(const void *x, int n_tokens, const int32_t
                                       const void *w_qkv, int hd, int k, void *q_act,
                                       void *k_cache, void *v_cache, void *stream);
 
+/* ------------------------------------------------------------------------
+ * jano_random_scores -- scores of the random-masking ablation.  Pages: ko
+ * technical summary, section 4 "Ablation Study" (random masking at a
+ * similar speed-up against Jano's convergence-aware levels).  Classifying
+ * these scores with jano_classify gives a level map with the same level
+ * counts as Jano's, assigned at random:
+ *
+ *   scores[b] = (r_{b+1} >> 40) * 2^-24,  r_i = output i of splitmix64 seeded with seed
+ *
+ * (splitmix64: Steele, Lea and Flood 2014; r_i is the 64-bit finaliser of
+ * seed + i * 0x9E3779B97F4A7C15, so the map depends on the seed and the
+ * block count only).  Uniform in [0, 1) with 24-bit resolution; ties, which
+ * are rare, fall to the lower block index in jano_classify.
+ *
+ * scores  device fp32 [n_blocks].  n_blocks >= 1.
+ * ---------------------------------------------------------------------- */
+JANO_API jano_status jano_random_scores(int n_blocks, uint64_t seed, float *scores, void *stream);
+
 /* Synchronises `stream`, returns the first device-side error recorded on the
  * current device since the last call (JANO_OK if none) and clears it. */
 JANO_API jano_status jano_get_device_error(void *stream);

@@ -38,7 +38,7 @@ STATUS_NAMES = {0: "JANO_OK", 1: "JANO_EINVAL", 2: "JANO_ESHAPE", 3: "JANO_EALIG
                 7: "JANO_ETIMEOUT", 8: "JANO_ECUDA"}
 EXPORTS = ("jano_block_scores", "jano_classify", "jano_build_schedule_workspace_bytes",
            "jano_build_schedule", "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention",
-           "jano_gather_gemm", "jano_qkv_project",
+           "jano_gather_gemm", "jano_qkv_project", "jano_random_scores",
            "jano_get_device_error", "jano_status_str", "jano_version")
 
 
@@ -79,13 +79,14 @@ def lib() -> C.CDLL:
         L.jano_active_attention.argtypes = [P, P, P, P, i, i, i, i, f, P, P]
         L.jano_gather_gemm.argtypes = [P, i, P, i, P, i, i, P, P, i, P]
         L.jano_qkv_project.argtypes = [P, i, P, i, P, i, i, P, P, P, P]
+        L.jano_random_scores.argtypes = [i, C.c_uint64, P, P]
         L.jano_get_device_error.argtypes = [P]
         L.jano_status_str.argtypes = [i]
         L.jano_status_str.restype = C.c_char_p
         L.jano_version.argtypes = []
         for fn in ("jano_block_scores", "jano_classify", "jano_build_schedule",
                    "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention", "jano_get_device_error",
-                   "jano_gather_gemm", "jano_qkv_project", "jano_version"):
+                   "jano_gather_gemm", "jano_qkv_project", "jano_random_scores", "jano_version"):
             getattr(L, fn).restype = C.c_int
         _lib = L
     return _lib
@@ -182,6 +183,11 @@ def jano_qkv_project(x, n_tokens, idx, n_act, w_qkv, hd, k, q_act, k_cache, v_ca
         _dev(w_qkv, "w_qkv", torch.bfloat16), hd, k, _dev(q_act, "q_act", torch.bfloat16),
         _dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
         _stream(stream)))
+
+
+def jano_random_scores(n_blocks, seed, scores, stream=None):
+    _check("jano_random_scores", lib().jano_random_scores(
+        n_blocks, C.c_uint64(seed), _dev(scores, "scores", torch.float32), _stream(stream)))
 
 
 def jano_get_device_error(stream=None) -> int:
@@ -297,6 +303,15 @@ def qkv_project(x, idx, w_qkv, q_act, k_cache, v_cache, stream=None) -> None:
     N, k = x.shape
     hd = w_qkv.shape[0] // 3
     jano_qkv_project(x, N, idx, idx.numel(), w_qkv, hd, k, q_act, k_cache, v_cache, stream)
+
+
+def random_scores(n_blocks: int, seed: int, out=None, stream=None) -> torch.Tensor:
+    """Uniform scores of the random-masking ablation (classify them for a
+    random level map with the analyzer's level counts)."""
+    if out is None:
+        out = torch.empty(n_blocks, dtype=torch.float32, device="cuda")
+    jano_random_scores(n_blocks, seed, out, stream)
+    return out
 
 
 def device_error(stream=None) -> int:

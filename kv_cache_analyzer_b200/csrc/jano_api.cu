@@ -182,6 +182,11 @@ jano_status jano_qkv_project(const void* x, int n_tokens, const int32_t* idx, in
                                        static_cast<cudaStream_t>(stream)));
 }
 
+jano_status jano_random_scores(int n_blocks, uint64_t seed, float* scores, void* stream) {
+    if (n_blocks < 1 || !scores) return JANO_EINVAL;
+    return from_cuda(launch_random_scores(n_blocks, seed, scores, static_cast<cudaStream_t>(stream)));
+}
+
 jano_status jano_get_device_error(void* stream) {
     int* err = device_error_word();
     if (!err) return JANO_ECUDA;

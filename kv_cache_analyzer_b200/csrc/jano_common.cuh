@@ -59,6 +59,7 @@ cudaError_t launch_projection(const void* x, int n_x, const int32_t* gather, int
                               int n, int k, int n_seg, const ProjSeg* segs, int* err,
                               cudaStream_t st);
 int projection_tile_n(int n, int seg_w, int n_seg);
+cudaError_t launch_random_scores(int n, uint64_t seed, float* scores, cudaStream_t st);
 
 namespace ptx {
 

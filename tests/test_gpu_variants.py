@@ -1,0 +1,54 @@
+"""GPU parity of the method variants next to the hot path: the random-masking
+ablation's scores and level maps (bit-exact: counter-based generator and
+integer ranks) and the Static refresh period of the pages' example (every
+5th step), through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def J():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from kv_cache_analyzer_b200 import build
+    build.build()
+    import kv_cache_analyzer_b200 as j
+    j.lib()
+    return j
+
+
+@pytest.mark.parametrize("n,seed", [(1, 0), (1000, 7), (8190, 2**63 + 5), (19320, 123456789)])
+def test_random_scores_bit_exact(J, n, seed):
+    got = J.random_scores(n, seed).cpu().numpy()
+    np.testing.assert_array_equal(got.view(np.uint32), oracle.random_scores(n, seed).view(np.uint32))
+
+
+@pytest.mark.parametrize("n,fa,fs", [(19320, 0.25, 0.45), (4096, 0.30, 0.40), (257, 0.35, 0.65)])
+def test_random_level_map_bit_exact_with_jano_counts(J, n, fa, fs):
+    lv = J.classify(J.random_scores(n, 42), fa, fs).cpu().numpy()
+    assert J.device_error() == 0
+    ref = oracle.classify(oracle.random_scores(n, 42), fa, fs)
+    np.testing.assert_array_equal(lv, ref)
+    n_a, n_s = oracle.level_counts(n, fa, fs)
+    assert (lv == 3).sum() == n_a and (lv == 1).sum() == n_s
+    # a different seed moves the levels, not their counts
+    lv2 = J.classify(J.random_scores(n, 43), fa, fs).cpu().numpy()
+    assert (lv2 == 3).sum() == n_a and not np.array_equal(lv, lv2)
+
+
+def test_schedule_static_every_5th_step_bit_exact(J):
+    g = np.random.default_rng(9)
+    F, H, W = 3, 12, 14
+    lv = g.integers(1, 4, size=F * 6 * 7).astype(np.uint8)
+    sched = J.Schedule(50, 5, 5, 2, 5)
+    geom = J.Geometry(F, H, W, (1, 2, 2), (1, 2, 2))
+    off, idx, tl = J.build_schedule(torch.from_numpy(lv).cuda(), geom, sched)
+    assert J.device_error() == 0
+    roff, ridx, rtl = oracle.build_schedule(lv, (F, H, W), (1, 2, 2), (1, 2, 2), 50, 5, 5, 2, 5)
+    np.testing.assert_array_equal(off.cpu().numpy(), roff)
+    np.testing.assert_array_equal(idx.cpu().numpy()[: roff[-1]], ridx)
+    np.testing.assert_array_equal(tl.cpu().numpy(), rtl)

@@ -509,3 +509,16 @@ def test_random_level_map_keeps_the_level_counts():
     lv = oracle.classify(oracle.random_scores(n, 7), 0.25, 0.45)
     n_a, n_s = oracle.level_counts(n, 0.25, 0.45)
     assert (lv == 3).sum() == n_a and (lv == 1).sum() == n_s and (lv == 2).sum() == n - n_a - n_s
+
+
+def test_schedule_closed_form_counts_static_every_5th_step():
+    # the page's example period for Level 1 ("e.g. every 5th step"): 50 steps,
+    # warm-up 5, cool-down 5, Moderate every 2, Static every 5 -> per token
+    # Active 40 + 10, Moderate 20 + 10, Static 8 + 10 refreshes
+    gen = np.random.default_rng(5)
+    bl = gen.integers(1, 4, size=6 * 7).astype(np.uint8)
+    off, idx, tl = oracle.build_schedule(bl, (1, 12, 14), (1, 2, 2), (1, 2, 2), 50, 5, 5, 2, 5)
+    counts = np.bincount(idx, minlength=bl.size)
+    np.testing.assert_array_equal(counts[bl == 3], 50)
+    np.testing.assert_array_equal(counts[bl == 2], 30)
+    np.testing.assert_array_equal(counts[bl == 1], 18)
