@@ -50,6 +50,7 @@ def _load():
         P = C.c_void_p
         i, d, f, ll = C.c_int, C.c_double, C.c_float, C.c_longlong
         lib.oracle_block_scores.argtypes = [P, i, i, i, i, i, i, i, i, d, d, P]
+        lib.oracle_block_scores_literal.argtypes = [P, i, i, i, i, i, i, i, i, d, d, P]
         lib.oracle_level_counts.argtypes = [i, f, f, P, P]
         lib.oracle_classify.argtypes = [P, i, f, f, P]
         lib.oracle_build_schedule.argtypes = [P, i, i, i, i, i, i, i, i, i,
@@ -60,7 +61,7 @@ def _load():
         lib.oracle_splitmix64.argtypes = [C.c_uint64, i, P]
         lib.oracle_splitmix64.restype = None
         lib.oracle_random_scores.argtypes = [i, C.c_uint64, P]
-        for fn in ("oracle_block_scores", "oracle_level_counts", "oracle_classify",
+        for fn in ("oracle_block_scores", "oracle_block_scores_literal", "oracle_level_counts", "oracle_classify",
                    "oracle_build_schedule", "oracle_kv_scatter", "oracle_active_attention",
                    "oracle_gather_gemm", "oracle_random_scores"):
             getattr(lib, fn).restype = C.c_int
@@ -85,6 +86,19 @@ def block_scores(lat, block, w_temporal=0.5, w_spatial=0.5):
     nB = (-(-F // bf)) * (-(-H // bh)) * (-(-W // bw))
     out = np.empty(nB, dtype=np.float64)
     _check("oracle_block_scores", _load().oracle_block_scores(
+        _ptr(lat), K1 - 1, Cc, F, H, W, bf, bh, bw, w_temporal, w_spatial, _ptr(out)))
+    return out
+
+
+def block_scores_literal(lat, block, w_temporal=0.5, w_spatial=0.5):
+    """The literal reading: second differences over the steps of the temporal
+    and spatial gradients.  lat fp32 [K+1][C][F][H][W] -> fp64 scores."""
+    lat = np.ascontiguousarray(lat, dtype=np.float32)
+    K1, Cc, F, H, W = lat.shape
+    bf, bh, bw = block
+    nB = (-(-F // bf)) * (-(-H // bh)) * (-(-W // bw))
+    out = np.empty(nB, dtype=np.float64)
+    _check("oracle_block_scores_literal", _load().oracle_block_scores_literal(
         _ptr(lat), K1 - 1, Cc, F, H, W, bf, bh, bw, w_temporal, w_spatial, _ptr(out)))
     return out
 

@@ -382,3 +382,73 @@ int oracle_random_scores(int n, uint64_t seed, float *scores)
     free(r);
     return OR_OK;
 }
+
+/*
+ * The literal reading of the score (nl page, Methodologie 1
+ * "Implementatie": the analyzer computes the second-order differences of
+ * the temporal and spatial gradients over the first steps).  Per element p
+ * and step k = 1..K-1, with the forward gradients of snapshot j
+ *
+ *   G_f(j) = D_f x_j(p),  G_h(j) = D_h x_j(p),  G_w(j) = D_w x_j(p)
+ *
+ * (0 where the neighbour lies outside the tensor) and their second
+ * difference over the steps, Delta2 G(k) = G(k+1) - 2 G(k) + G(k-1):
+ *
+ *   S_b = mean over k and p in P_b of
+ *           w_t |Delta2 G_f(k)| + w_s sqrt(Delta2 G_h(k)^2 + Delta2 G_w(k)^2)
+ *
+ * Computed in that order (the gradients of the three snapshots first, then
+ * their second difference), fp64.  Same blocks, layout and edge rules as
+ * oracle_block_scores.
+ */
+static double or_grad(const float *x, size_t p, int on, size_t step)
+{
+    return on ? (double)x[p + step] - (double)x[p] : 0.0;
+}
+
+int oracle_block_scores_literal(const float *lat, int K, int C, int F, int H, int W,
+                                int bf, int bh, int bw, double w_t, double w_s,
+                                double *scores)
+{
+    if (!lat || !scores || K < 2 || C < 1 || F < 1 || H < 1 || W < 1 ||
+        bf < 1 || bh < 1 || bw < 1)
+        return OR_EINVAL;
+    const int nBf = ceil_div(F, bf), nBh = ceil_div(H, bh), nBw = ceil_div(W, bw);
+    const size_t nB = (size_t)nBf * nBh * nBw;
+    const size_t plane = (size_t)H * W;
+    const size_t vol = (size_t)F * plane;
+    const size_t snap = (size_t)C * vol;
+
+    double *sum = (double *)calloc(nB, sizeof(double));
+    double *cnt = (double *)calloc(nB, sizeof(double));
+    if (!sum || !cnt) { free(sum); free(cnt); return OR_ENOMEM; }
+
+    for (int k = 1; k <= K - 1; ++k) {
+        const float *xs[3] = {lat + (size_t)(k - 1) * snap, lat + (size_t)k * snap,
+                              lat + (size_t)(k + 1) * snap};
+        for (int c = 0; c < C; ++c)
+            for (int f = 0; f < F; ++f)
+                for (int h = 0; h < H; ++h)
+                    for (int w = 0; w < W; ++w) {
+                        const size_t p = (size_t)c * vol + (size_t)f * plane + (size_t)h * W + w;
+                        double gf[3], gh[3], gw[3];
+                        for (int j = 0; j < 3; ++j) {
+                            gf[j] = or_grad(xs[j], p, f + 1 < F, plane);
+                            gh[j] = or_grad(xs[j], p, h + 1 < H, (size_t)W);
+                            gw[j] = or_grad(xs[j], p, w + 1 < W, 1);
+                        }
+                        const double d2f = gf[2] - 2.0 * gf[1] + gf[0];
+                        const double d2h = gh[2] - 2.0 * gh[1] + gh[0];
+                        const double d2w = gw[2] - 2.0 * gw[1] + gw[0];
+                        const double term = w_t * fabs(d2f) + w_s * sqrt(d2h * d2h + d2w * d2w);
+                        const size_t b = ((size_t)(f / bf) * nBh + (size_t)(h / bh)) * nBw + (size_t)(w / bw);
+                        sum[b] += term;
+                        cnt[b] += 1.0;
+                    }
+    }
+    for (size_t b = 0; b < nB; ++b)
+        scores[b] = sum[b] / cnt[b];
+    free(sum);
+    free(cnt);
+    return OR_OK;
+}

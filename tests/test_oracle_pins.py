@@ -522,3 +522,66 @@ def test_schedule_closed_form_counts_static_every_5th_step():
     np.testing.assert_array_equal(counts[bl == 3], 50)
     np.testing.assert_array_equal(counts[bl == 2], 30)
     np.testing.assert_array_equal(counts[bl == 1], 18)
+
+
+# ---------------------------------------------------------------- literal score reading
+def _grad(x, axis):
+    """Forward difference along `axis`, 0 at the last index (numpy)."""
+    g = np.zeros_like(x)
+    sl_lo = [slice(None)] * x.ndim
+    sl_hi = [slice(None)] * x.ndim
+    sl_lo[axis] = slice(0, -1)
+    sl_hi[axis] = slice(1, None)
+    g[tuple(sl_lo)] = x[tuple(sl_hi)] - x[tuple(sl_lo)]
+    return g
+
+
+def test_literal_score_equals_gradients_of_the_second_difference():
+    # Delta2 and the forward differences are linear and commute, so the
+    # literal score (gradients first, then the second difference over steps)
+    # equals the gradient magnitudes of the second difference, computed here
+    # by numpy in the other order and reduced per block by reshaping
+    gen = np.random.default_rng(41)
+    lat = gen.standard_normal((5, 3, 4, 8, 12)).astype(np.float32)
+    x = lat.astype(np.float64)
+    d2 = x[2:] - 2 * x[1:-1] + x[:-2]                        # [K-1][C][F][H][W]
+    term = 0.5 * np.abs(_grad(d2, 2)) + 0.5 * np.sqrt(_grad(d2, 3) ** 2 + _grad(d2, 4) ** 2)
+    per = term.reshape(3, 3, 4, 2, 4, 3, 4).transpose(2, 3, 5, 0, 1, 4, 6).reshape(4 * 2 * 3, -1)
+    np.testing.assert_allclose(oracle.block_scores_literal(lat, (1, 4, 4)), per.mean(axis=1), rtol=1e-12)
+
+
+def test_literal_score_is_zero_for_steps_affine_in_k():
+    # x_k = a(p) + k b(p): every gradient is affine in k, its second difference 0
+    gen = np.random.default_rng(42)
+    a, b = gen.standard_normal((2, 2, 3, 8, 8))
+    lat = np.stack([a + k * b for k in range(6)]).astype(np.float32)
+    np.testing.assert_allclose(oracle.block_scores_literal(lat, (1, 4, 4)), 0.0, atol=2e-5)
+
+
+def test_literal_score_closed_forms_for_quadratic_steps():
+    # x_k = k^2 c(p): Delta2 of any gradient of x is 2 * (gradient of c).
+    # c = alpha * h: spatial term 2|alpha| except the last row (0);
+    # c = beta * f: temporal term 2|beta| except the last frame (0)
+    K1, F, H, W = 5, 3, 8, 8
+    alpha, beta = 0.75, -1.25
+    hh = np.arange(H, dtype=np.float64)[None, None, :, None] * np.ones((1, F, 1, W))
+    ff = np.arange(F, dtype=np.float64)[None, :, None, None] * np.ones((1, 1, H, W))
+    for c_field, expect in ((alpha * hh, "h"), (beta * ff, "f")):
+        lat = np.stack([k * k * c_field for k in range(K1)]).astype(np.float32)
+        got = oracle.block_scores_literal(lat, (1, 4, 4), 0.5, 0.5).reshape(F, 2, 2)
+        if expect == "h":
+            # rows 0..3 of block row 0 all interior; block row 1 has rows 4..7, row 7 is the edge
+            np.testing.assert_allclose(got[:, 0, :], 0.5 * 2 * abs(alpha), rtol=1e-6)
+            np.testing.assert_allclose(got[:, 1, :], 0.5 * 2 * abs(alpha) * 3 / 4, rtol=1e-6)
+        else:
+            np.testing.assert_allclose(got[:-1], 0.5 * 2 * abs(beta), rtol=1e-6)
+            np.testing.assert_allclose(got[-1], 0.0, atol=1e-12)
+
+
+def test_literal_and_additive_readings_differ():
+    # the two readings are different scores (the additive one has |Delta2 x|
+    # and first-order gradients): a plain spatial ramp constant over the steps
+    # scores 0 under the literal reading but not under the additive one
+    hh = np.arange(8, dtype=np.float32)[None, None, None, :, None] * np.ones((6, 1, 2, 8, 8), np.float32)
+    assert np.all(oracle.block_scores_literal(hh, (1, 4, 4)) == 0.0)
+    assert np.all(oracle.block_scores(hh, (1, 4, 4))[:2] > 0.0)
