@@ -105,6 +105,24 @@ JANO_API jano_status jano_block_scores(const float *lat, int K, int C, const jan
                               void *stream);
 
 /* ------------------------------------------------------------------------
+ * jano_block_scores_literal -- the literal reading of the score: the
+ * second-order differences over the steps of the temporal and spatial
+ * gradients (nl technical summary, Methodologie 1 "Implementatie").
+ *
+ *   S_b = mean over k=1..K-1 and every (c,f,h,w) in block b of
+ *         w_temporal |D2 D_f x_k| + w_spatial sqrt((D2 D_h x_k)^2 + (D2 D_w x_k)^2)
+ *   D2 y_k = y_{k+1} - 2 y_k + y_{k-1}
+ *
+ * with the forward differences and edge rules of jano_block_scores.  It
+ * differs from jano_block_scores (which adds |D2 x| to first-order
+ * gradients) only in the formula; arguments, layout, limits and errors are
+ * the same.  Deterministic.
+ * ---------------------------------------------------------------------- */
+JANO_API jano_status jano_block_scores_literal(const float *lat, int K, int C, const jano_geom *g,
+                                               float w_temporal, float w_spatial, float *scores,
+                                               void *stream);
+
+/* ------------------------------------------------------------------------
  * jano_classify -- three convergence levels (Level 1 Static, 2 Moderate,
  * 3 Active).  Pages: nl technical summary, Methodologie 1 "Resultaat";
  * zh 2.2 item 1; ko 2.B.

@@ -36,7 +36,7 @@ library_path = os.environ.get("JANO_LIBRARY") or os.path.join(_HERE, "libjano.so
 STATUS_NAMES = {0: "JANO_OK", 1: "JANO_EINVAL", 2: "JANO_ESHAPE", 3: "JANO_EALIGN",
                 4: "JANO_EUNSUPPORTED", 5: "JANO_ENONFINITE", 6: "JANO_EINDEX",
                 7: "JANO_ETIMEOUT", 8: "JANO_ECUDA"}
-EXPORTS = ("jano_block_scores", "jano_classify", "jano_build_schedule_workspace_bytes",
+EXPORTS = ("jano_block_scores", "jano_block_scores_literal", "jano_classify", "jano_build_schedule_workspace_bytes",
            "jano_build_schedule", "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention",
            "jano_gather_gemm", "jano_qkv_project", "jano_random_scores",
            "jano_get_device_error", "jano_status_str", "jano_version")
@@ -70,6 +70,7 @@ def lib() -> C.CDLL:
         P, i, f, z = C.c_void_p, C.c_int, C.c_float, C.c_size_t
         G, S = C.POINTER(jano_geom), C.POINTER(jano_sched_cfg)
         L.jano_block_scores.argtypes = [P, i, i, G, f, f, P, P]
+        L.jano_block_scores_literal.argtypes = [P, i, i, G, f, f, P, P]
         L.jano_classify.argtypes = [P, i, f, f, P, P]
         L.jano_build_schedule_workspace_bytes.argtypes = [G]
         L.jano_build_schedule_workspace_bytes.restype = z
@@ -84,7 +85,7 @@ def lib() -> C.CDLL:
         L.jano_status_str.argtypes = [i]
         L.jano_status_str.restype = C.c_char_p
         L.jano_version.argtypes = []
-        for fn in ("jano_block_scores", "jano_classify", "jano_build_schedule",
+        for fn in ("jano_block_scores", "jano_block_scores_literal", "jano_classify", "jano_build_schedule",
                    "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention", "jano_get_device_error",
                    "jano_gather_gemm", "jano_qkv_project", "jano_random_scores", "jano_version"):
             getattr(L, fn).restype = C.c_int
@@ -118,6 +119,12 @@ def _check(fn: str, code: int) -> None:
 # ---------------------------------------------------------------- C ABI mirror
 def jano_block_scores(lat, K, C_, geom, w_temporal, w_spatial, scores, stream=None):
     _check("jano_block_scores", lib().jano_block_scores(
+        _dev(lat, "lat", torch.float32), K, C_, C.byref(geom), w_temporal, w_spatial,
+        _dev(scores, "scores", torch.float32), _stream(stream)))
+
+
+def jano_block_scores_literal(lat, K, C_, geom, w_temporal, w_spatial, scores, stream=None):
+    _check("jano_block_scores_literal", lib().jano_block_scores_literal(
         _dev(lat, "lat", torch.float32), K, C_, C.byref(geom), w_temporal, w_spatial,
         _dev(scores, "scores", torch.float32), _stream(stream)))
 
@@ -245,6 +252,16 @@ def block_scores(lat: torch.Tensor, geom: Geometry, w_temporal=0.5, w_spatial=0.
     if out is None:
         out = torch.empty(geom.n_blocks, dtype=torch.float32, device=lat.device)
     jano_block_scores(lat, K1 - 1, Cc, geom.c(), w_temporal, w_spatial, out, stream)
+    return out
+
+
+def block_scores_literal(lat: torch.Tensor, geom: Geometry, w_temporal=0.5, w_spatial=0.5,
+                         out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The literal reading: second differences over the steps of the gradients."""
+    K1, Cc = lat.shape[0], lat.shape[1]
+    if out is None:
+        out = torch.empty(geom.n_blocks, dtype=torch.float32, device=lat.device)
+    jano_block_scores_literal(lat, K1 - 1, Cc, geom.c(), w_temporal, w_spatial, out, stream)
     return out
 
 

@@ -22,6 +22,12 @@
 // fixed order (deterministic, no atomics).
 // Every byte of the latent is read from HBM once; neighbour rows and frames
 // come back from L2.
+//
+// The literal reading (second differences over the steps of the gradients,
+//   w_t |D2 D_f x| + w_s sqrt((D2 D_h x)^2 + (D2 D_w x)^2),  D2 y = y_{k+1} - 2y_k + y_{k-1})
+// runs the same pipeline with box B widened to snapshots 0..K: since D2 and
+// the forward differences commute, a thread forms D2 x at its element and at
+// the f+1, h+1, w+1 neighbours and takes their differences.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -103,6 +109,20 @@ __device__ __forceinline__ void named_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+__device__ __forceinline__ float4 d2_of(const float* A, int o, int kA) {
+    const float4 m = *reinterpret_cast<const float4*>(A + o - kA);
+    const float4 z = *reinterpret_cast<const float4*>(A + o);
+    const float4 p = *reinterpret_cast<const float4*>(A + o + kA);
+    return make_float4(p.x - 2.f * z.x + m.x, p.y - 2.f * z.y + m.y, p.z - 2.f * z.z + m.z,
+                       p.w - 2.f * z.w + m.w);
+}
+
+__device__ __forceinline__ float lit_term(float gf, float gh, float gw, float w_t, float w_s) {
+    return w_t * fabsf(gf) + w_s * ptx::sqrt_approx(fmaf(gh, gh, gw * gw));
+}
+
+// kLit: the literal reading (see the file comment).
+template <bool kLit>
 __global__ void __launch_bounds__(1024)
 analyzer_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 AGeo g, float* __restrict__ scores, int* err) {
@@ -151,7 +171,7 @@ analyzer_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     ptx::mbar_arrive_expect_tx(full(slot), g.bytesA + (has_next ? g.bytesB : 0));
                     tma_load_5d(dst, &tmA, full(slot), w0, h0, f0, c, 0);
                     if (has_next)
-                        tma_load_5d(dst + g.offB, &tmB, full(slot), w0, h0, f0 + g.bf, c, 1);
+                        tma_load_5d(dst + g.offB, &tmB, full(slot), w0, h0, f0 + g.bf, c, kLit ? 0 : 1);
                     last[slot] = phase;
                     if (++slot == S) { slot = 0; phase ^= 1; }
                 }
@@ -179,6 +199,12 @@ analyzer_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     const int o_xp = o_x0 + g.bf * rowsA * LA;
     const int o_nh = o_x0 + LA;
     const int o_nf = fr + 1 < g.bf ? o_x0 + rowsA * LA : g.offB / 4 + ((k - 1) * g.bh + hr) * g.Wc + wr;
+    // literal reading: snapshot stride inside box A, and the f+1 neighbour at
+    // snapshot k with its own snapshot stride (box B then holds 0..K)
+    const int kA = g.bf * rowsA * LA;
+    const bool nf_in_A = fr + 1 < g.bf;
+    const int o_nf_lit = nf_in_A ? o_x0 + rowsA * LA : g.offB / 4 + (k * g.bh + hr) * g.Wc + wr;
+    const int kF_lit = nf_in_A ? kA : g.bh * g.Wc;
     int slot = 0, phase = 0;                       // ring position, advanced incrementally
     for (int u = blockIdx.x; u < g.n_units; u += gridDim.x) {
         const int wc = u % g.n_wc;
@@ -196,22 +222,39 @@ analyzer_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const bool ready = bounded_wait(full(slot), (uint32_t)phase, err, abort);
             if (ready && act) {
                 const float* A = reinterpret_cast<const float*>(gbase + (size_t)slot * g.stage_bytes);
+                if constexpr (kLit) {
 #pragma unroll
-                for (int v = 0; v < kVec; ++v) {
-                    const float4 x0 = *reinterpret_cast<const float4*>(A + o_x0 + 4 * v);
-                    const float4 xm = *reinterpret_cast<const float4*>(A + o_xm + 4 * v);
-                    const float4 xp = *reinterpret_cast<const float4*>(A + o_xp + 4 * v);
-                    const float4 nh = has_h ? *reinterpret_cast<const float4*>(A + o_nh + 4 * v) : x0;
-                    const float4 nf = has_f ? *reinterpret_cast<const float4*>(A + o_nf + 4 * v) : x0;
-                    // w+1 neighbour of the 4th element; zero-filled beyond the tensor, and the
-                    // difference is dropped there (w + 4v + 4 >= W)
-                    const float nx = A[o_x0 + 4 * v + 4];
-                    const float nw = (w + 4 * v + 4 < g.W) ? nx : x0.w;
-                    float* a = acc + 4 * v;
-                    a[0] += term(xp.x - 2.f * x0.x + xm.x, nf.x - x0.x, nh.x - x0.x, x0.y - x0.x, g.w_t, g.w_s);
-                    a[1] += term(xp.y - 2.f * x0.y + xm.y, nf.y - x0.y, nh.y - x0.y, x0.z - x0.y, g.w_t, g.w_s);
-                    a[2] += term(xp.z - 2.f * x0.z + xm.z, nf.z - x0.z, nh.z - x0.z, x0.w - x0.z, g.w_t, g.w_s);
-                    a[3] += term(xp.w - 2.f * x0.w + xm.w, nf.w - x0.w, nh.w - x0.w, nw - x0.w, g.w_t, g.w_s);
+                    for (int v = 0; v < kVec; ++v) {
+                        const float4 d = d2_of(A, o_x0 + 4 * v, kA);
+                        const float4 dh = has_h ? d2_of(A, o_nh + 4 * v, kA) : d;
+                        const float4 df = has_f ? d2_of(A, o_nf_lit + 4 * v, kF_lit) : d;
+                        // w+1 neighbour of the 4th element (dropped past the tensor)
+                        const int ow = o_x0 + 4 * v + 4;
+                        const float dw = (w + 4 * v + 4 < g.W) ? A[ow + kA] - 2.f * A[ow] + A[ow - kA] : d.w;
+                        float* a = acc + 4 * v;
+                        a[0] += lit_term(df.x - d.x, dh.x - d.x, d.y - d.x, g.w_t, g.w_s);
+                        a[1] += lit_term(df.y - d.y, dh.y - d.y, d.z - d.y, g.w_t, g.w_s);
+                        a[2] += lit_term(df.z - d.z, dh.z - d.z, d.w - d.z, g.w_t, g.w_s);
+                        a[3] += lit_term(df.w - d.w, dh.w - d.w, dw - d.w, g.w_t, g.w_s);
+                    }
+                } else {
+#pragma unroll
+                    for (int v = 0; v < kVec; ++v) {
+                        const float4 x0 = *reinterpret_cast<const float4*>(A + o_x0 + 4 * v);
+                        const float4 xm = *reinterpret_cast<const float4*>(A + o_xm + 4 * v);
+                        const float4 xp = *reinterpret_cast<const float4*>(A + o_xp + 4 * v);
+                        const float4 nh = has_h ? *reinterpret_cast<const float4*>(A + o_nh + 4 * v) : x0;
+                        const float4 nf = has_f ? *reinterpret_cast<const float4*>(A + o_nf + 4 * v) : x0;
+                        // w+1 neighbour of the 4th element; zero-filled beyond the tensor, and the
+                        // difference is dropped there (w + 4v + 4 >= W)
+                        const float nx = A[o_x0 + 4 * v + 4];
+                        const float nw = (w + 4 * v + 4 < g.W) ? nx : x0.w;
+                        float* a = acc + 4 * v;
+                        a[0] += term(xp.x - 2.f * x0.x + xm.x, nf.x - x0.x, nh.x - x0.x, x0.y - x0.x, g.w_t, g.w_s);
+                        a[1] += term(xp.y - 2.f * x0.y + xm.y, nf.y - x0.y, nh.y - x0.y, x0.z - x0.y, g.w_t, g.w_s);
+                        a[2] += term(xp.z - 2.f * x0.z + xm.z, nf.z - x0.z, nh.z - x0.z, x0.w - x0.z, g.w_t, g.w_s);
+                        a[3] += term(xp.w - 2.f * x0.w + xm.w, nf.w - x0.w, nh.w - x0.w, nw - x0.w, g.w_t, g.w_s);
+                    }
                 }
             }
             __syncwarp();
@@ -269,7 +312,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // Unit width, ring depth and shared memory for a geometry; false if unsupported.
-bool plan(const jano_geom& gm, int K, int C, AGeo& a) {
+bool plan(const jano_geom& gm, int K, int C, bool literal, AGeo& a) {
     a.K = K; a.C = C; a.F = gm.F; a.H = gm.H; a.W = gm.W;
     a.bf = gm.bf; a.bh = gm.bh; a.bw = gm.bw;
     a.nBh = (gm.H + gm.bh - 1) / gm.bh;
@@ -292,7 +335,7 @@ bool plan(const jano_geom& gm, int K, int C, AGeo& a) {
     a.NP = R * (Wc / (4 * kVec));
     a.NC = (a.NP * (K - 1) + 31) / 32 * 32;
     a.bytesA = a.LA * (gm.bh + 1) * gm.bf * (K + 1) * 4;
-    a.bytesB = Wc * gm.bh * (K - 1) * 4;
+    a.bytesB = Wc * gm.bh * (literal ? K + 1 : K - 1) * 4;   // snapshots 0..K or 1..K-1
     a.offB = (a.bytesA + 127) / 128 * 128;
     a.stage_bytes = (a.offB + a.bytesB + 127) / 128 * 128;
     const long long fixed = (long long)(K - 1) * R * Wc * 4 + 128 + 16;   // red + slack + abort
@@ -316,16 +359,16 @@ bool plan(const jano_geom& gm, int K, int C, AGeo& a) {
 
 }  // namespace
 
-bool analyzer_supported(const jano_geom& g, int K, int C) {
+bool analyzer_supported(const jano_geom& g, int K, int C, bool literal) {
     AGeo a;
-    return plan(g, K, C, a);
+    return plan(g, K, C, literal, a);
 }
 
 cudaError_t launch_block_scores(const float* lat, int K, int C, const jano_geom& gm,
-                                float w_t, float w_s, float* scores, int* err,
+                                float w_t, float w_s, bool literal, float* scores, int* err,
                                 cudaStream_t st) {
     AGeo a;
-    if (!plan(gm, K, C, a)) return cudaErrorInvalidValue;
+    if (!plan(gm, K, C, literal, a)) return cudaErrorInvalidValue;
     a.w_t = w_t;
     a.w_s = w_s;
     auto fn = encode_fn();
@@ -337,7 +380,8 @@ cudaError_t launch_block_scores(const float* lat, int K, int C, const jano_geom&
                                    (cuuint64_t)C * gm.F * gm.H * gm.W * 4};
     const cuuint32_t boxA[5] = {(cuuint32_t)a.Wc + 4, (cuuint32_t)gm.bh + 1, (cuuint32_t)gm.bf, 1,
                                 (cuuint32_t)K + 1};
-    const cuuint32_t boxB[5] = {(cuuint32_t)a.Wc, (cuuint32_t)gm.bh, 1, 1, (cuuint32_t)K - 1};
+    const cuuint32_t boxB[5] = {(cuuint32_t)a.Wc, (cuuint32_t)gm.bh, 1, 1,
+                                (cuuint32_t)(literal ? K + 1 : K - 1)};
     const cuuint32_t es[5] = {1, 1, 1, 1, 1};
     CUtensorMap mA, mB;
     if (fn(&mA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, const_cast<float*>(lat), dims, strides, boxA, es,
@@ -349,15 +393,15 @@ cudaError_t launch_block_scores(const float* lat, int K, int C, const jano_geom&
         return cudaErrorInvalidValue;
 
     const size_t smem = (size_t)a.smem;
-    static unsigned long long done_mask = 0;   // per-device shared-memory opt-in
+    static unsigned long long done_mask[2] = {0, 0};   // per-device shared-memory opt-in
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (dev >= 64 || !(done_mask & (1ull << dev))) {
-        cudaError_t e = cudaFuncSetAttribute(analyzer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             224 * 1024);
+    if (dev >= 64 || !(done_mask[literal] & (1ull << dev))) {
+        cudaError_t e = cudaFuncSetAttribute(literal ? analyzer_kernel<true> : analyzer_kernel<false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 224 * 1024);
         if (e != cudaSuccess) return e;
-        if (dev < 64) done_mask |= 1ull << dev;
+        if (dev < 64) done_mask[literal] |= 1ull << dev;
     }
     const int threads = a.NC + 32;
     // resident CTAs per SM: shared memory (228 KB, 1 KB reserved per CTA) and threads
@@ -365,7 +409,8 @@ cudaError_t launch_block_scores(const float* lat, int K, int C, const jano_geom&
     if (per_sm > 2048 / threads) per_sm = 2048 / threads;
     if (per_sm < 1) per_sm = 1;
     const int grid = a.n_units < per_sm * sms ? a.n_units : per_sm * sms;
-    analyzer_kernel<<<grid, threads, smem, st>>>(mA, mB, a, scores, err);
+    if (literal) analyzer_kernel<true><<<grid, threads, smem, st>>>(mA, mB, a, scores, err);
+    else analyzer_kernel<false><<<grid, threads, smem, st>>>(mA, mB, a, scores, err);
     return cudaGetLastError();
 }
 

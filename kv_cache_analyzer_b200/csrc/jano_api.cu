@@ -52,9 +52,9 @@ using namespace jano;
 
 extern "C" {
 
-jano_status jano_block_scores(const float* lat, int K, int C, const jano_geom* g,
-                              float w_temporal, float w_spatial, float* scores,
-                              void* stream) {
+namespace {
+jano_status block_scores_impl(const float* lat, int K, int C, const jano_geom* g, float w_temporal,
+                              float w_spatial, bool literal, float* scores, void* stream) {
     if (!lat || !scores) return JANO_EINVAL;
     if (K < 2 || C < 1) return JANO_EINVAL;
     if (!std::isfinite(w_temporal) || !std::isfinite(w_spatial)) return JANO_EINVAL;
@@ -62,11 +62,24 @@ jano_status jano_block_scores(const float* lat, int K, int C, const jano_geom* g
     if (gs != JANO_OK) return gs;
     if (g->W % 4) return JANO_EUNSUPPORTED;
     if (!aligned16(lat)) return JANO_EALIGN;
-    if (!analyzer_supported(*g, K, C)) return JANO_EUNSUPPORTED;
+    if (!analyzer_supported(*g, K, C, literal)) return JANO_EUNSUPPORTED;
     int* err = device_error_word();
     if (!err) return JANO_ECUDA;
-    return from_cuda(launch_block_scores(lat, K, C, *g, w_temporal, w_spatial, scores, err,
+    return from_cuda(launch_block_scores(lat, K, C, *g, w_temporal, w_spatial, literal, scores, err,
                                          static_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+
+jano_status jano_block_scores(const float* lat, int K, int C, const jano_geom* g,
+                              float w_temporal, float w_spatial, float* scores,
+                              void* stream) {
+    return block_scores_impl(lat, K, C, g, w_temporal, w_spatial, false, scores, stream);
+}
+
+jano_status jano_block_scores_literal(const float* lat, int K, int C, const jano_geom* g,
+                                      float w_temporal, float w_spatial, float* scores,
+                                      void* stream) {
+    return block_scores_impl(lat, K, C, g, w_temporal, w_spatial, true, scores, stream);
 }
 
 jano_status jano_classify(const float* scores, int n_blocks, float frac_active,

@@ -26,12 +26,12 @@ int* device_error_word();   // address of this device's error word (host)
 // Launchers implemented by the kernel translation units.  They assume the
 // arguments were validated by the exported entry points.
 cudaError_t launch_block_scores(const float* lat, int K, int C, const jano_geom& g,
-                                float w_t, float w_s, float* scores, int* err,
+                                float w_t, float w_s, bool literal, float* scores, int* err,
                                 cudaStream_t st);
 cudaError_t launch_classify(const float* scores, int n, long long k_static,
                             long long k_active, uint8_t* levels, int* err,
                             cudaStream_t st);
-bool analyzer_supported(const jano_geom& g, int K, int C);
+bool analyzer_supported(const jano_geom& g, int K, int C, bool literal);
 size_t schedule_workspace_bytes(const jano_geom& g);
 cudaError_t launch_build_schedule(const uint8_t* block_levels, const jano_geom& g,
                                   const jano_sched_cfg& c, int32_t* offsets,

@@ -52,3 +52,36 @@ def test_schedule_static_every_5th_step_bit_exact(J):
     np.testing.assert_array_equal(off.cpu().numpy(), roff)
     np.testing.assert_array_equal(idx.cpu().numpy()[: roff[-1]], ridx)
     np.testing.assert_array_equal(tl.cpu().numpy(), rtl)
+
+
+# ---------------------------------------------------------------- literal score reading
+@pytest.mark.parametrize("name", ["tiny", "image", "small", "large"])
+def test_literal_scores_match_oracle(J, name):
+    """fp32 on the GPU, fp64 in the oracle.  The literal score takes
+    differences of second differences, whose fp32 rounding is absolute (a few
+    units of 2^-24 max|x|) while the scores of smooth content are small, so
+    the bound is 1e-5 |ref| + 2^-19 max|x| per block."""
+    import synth
+    from workloads import latent
+    w = synth.WORKLOADS[name]
+    lat = latent(name)
+    geom = J.Geometry(w.F, w.H, w.W, w.block, w.patch)
+    got = J.block_scores_literal(torch.from_numpy(lat).cuda(), geom).cpu().numpy()
+    assert J.device_error() == 0
+    ref = oracle.block_scores_literal(lat, w.block)
+    bound = 1e-5 * np.abs(ref) + 2.0 ** -19 * float(np.abs(lat).max())
+    assert np.all(np.abs(got - ref) <= bound), float(np.max(np.abs(got - ref) - bound))
+    again = J.block_scores_literal(torch.from_numpy(lat).cuda(), geom).cpu().numpy()
+    np.testing.assert_array_equal(got.view(np.uint32), again.view(np.uint32))
+
+
+@pytest.mark.parametrize("shape,block", [((3, 2, 3, 9, 12), (1, 4, 4)), ((4, 3, 5, 6, 8), (2, 3, 2)),
+                                         ((6, 1, 1, 16, 16), (1, 2, 2)), ((3, 1, 2, 4, 20), (1, 4, 8))])
+def test_literal_scores_edge_geometries(J, shape, block):
+    g = np.random.default_rng(sum(shape) + 1)
+    lat = g.standard_normal(shape).astype(np.float32)
+    K1, Cc, F, H, W = shape
+    got = J.block_scores_literal(torch.from_numpy(lat).cuda(), J.Geometry(F, H, W, block, (1, 1, 1))).cpu().numpy()
+    ref = oracle.block_scores_literal(lat, block)
+    bound = 1e-5 * np.abs(ref) + 2.0 ** -19 * float(np.abs(lat).max())
+    assert np.all(np.abs(got - ref) <= bound)
