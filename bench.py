@@ -285,7 +285,7 @@ def run_reference(args, w, rank, world):
 def run_gpu(args, w, rank, world, local_rank, dist):
     import torch
     import kv_cache_analyzer_b200 as J
-    from kv_cache_analyzer_b200.pipeline import HotPath, KERNELS_PER_STEP
+    from kv_cache_analyzer_b200.pipeline import HostStepper, HotPath, KERNELS_PER_STEP
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -353,17 +353,16 @@ def run_gpu(args, w, rank, world, local_rank, dist):
         host["q_act"] = host["q_act"][:n_act]; host["k_act"] = host["k_act"][:n_act]
         host["v_act"] = host["v_act"][:n_act]
         host_out = torch.empty(hp.out.shape, dtype=hp.out.dtype).pin_memory()
-        for _ in range(max(1, args.warmup)):
-            hp.step_from_host(step, host, host_out)
-        stream.synchronize()
-        barrier()
-        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s2.record(stream)
-        for _ in range(args.steps):
-            hp.step_from_host(step, host, host_out)
-        e2.record(stream)
+        own = {k: getattr(hp, k) for k in HostStepper.IN_KEYS + ("out",)}
+        stepper = HostStepper(hp, host, host_out)
+        stepper.run(step, max(1, args.warmup))
         torch.cuda.synchronize(dev)
         barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        stepper.run(step, args.steps, start=s2, end=e2)
+        torch.cuda.synchronize(dev)
+        barrier()
+        hp.use(own)
         e2e_ms = max_over_ranks(s2.elapsed_time(e2), dist, dev)
         e2e = {"value": whole_job_tflops(flops, world, e2e_ms / args.steps), "unit": "TFLOP/s",
                "h2d_bytes_per_step": HotPath.h2d_bytes(host),

@@ -80,6 +80,13 @@ class HotPath:
                             self.idx.numel(), self.token_levels, self.ws, self.ws_bytes, s)
         if ev[3] is not None: ev[3].record(s)
 
+    def use(self, bufs: dict):
+        """Point the step at another set of input/output buffers (keys lat,
+        field, q_act, k_act, v_act, out); the kernels take the pointers when
+        they are enqueued."""
+        for k, v in bufs.items():
+            setattr(self, k, v)
+
     def plan(self):
         """Run a1..a3 once and read the CSR offsets back (one D2H per generation)."""
         self.run_plan_kernels()
@@ -125,3 +132,73 @@ class HotPath:
     def h2d_bytes(host: dict) -> int:
         return sum(host[k].numel() * host[k].element_size()
                    for k in ("lat", "field", "q_act", "k_act", "v_act"))
+
+
+class HostStepper:
+    """End-to-end steps from pinned host memory, pipelined over three streams.
+
+    Every step copies its inputs (latent, field, q/k/v of the due tokens) in
+    from the pinned host buffers and its result (`out`) back to pinned host
+    memory.  Two device sets of those buffers alternate, so the inputs of
+    step i+1 are copied in (copy-in stream) and the result of step i-1 is
+    copied out (copy-out stream) while step i computes on the hot path's
+    stream; events order every reuse of a buffer.  The per-generation state
+    (scores, levels, schedule, KV cache) stays on the compute stream."""
+
+    IN_KEYS = ("lat", "field", "q_act", "k_act", "v_act")
+
+    def __init__(self, hp: HotPath, host: dict, host_out: torch.Tensor):
+        self.hp, self.host, self.host_out = hp, host, host_out
+        dev = hp.dev
+        self.h2d = torch.cuda.Stream(dev)
+        self.d2h = torch.cuda.Stream(dev)
+        self.sets = []
+        for _ in range(2):
+            b = {k: torch.empty(host[k].shape, dtype=host[k].dtype, device=dev) for k in self.IN_KEYS}
+            b["out"] = torch.zeros_like(hp.out)
+            self.sets.append(b)
+        ev = lambda: torch.cuda.Event()
+        self.ev_in = [ev(), ev()]      # the set's inputs have landed
+        self.ev_used = [ev(), ev()]    # the step on the set is done (inputs free, out final)
+        self.ev_out = [ev(), ev()]     # the set's out is back in host memory
+        self.used = [False, False]
+
+    def _copy_in(self, b: int):
+        s = self.h2d
+        if self.used[b]:
+            s.wait_event(self.ev_used[b])
+        with torch.cuda.stream(s):
+            for k in self.IN_KEYS:
+                self.sets[b][k].copy_(self.host[k], non_blocking=True)
+        self.ev_in[b].record(s)
+
+    def run(self, step: int, n_steps: int, start: torch.cuda.Event | None = None,
+            end: torch.cuda.Event | None = None):
+        """n_steps end-to-end steps of sampling step `step`; `start` / `end`
+        (optional) are recorded on the compute stream around all of them, with
+        the copy streams ordered inside."""
+        cs = self.hp.stream
+        if start is not None:
+            start.record(cs)
+            self.h2d.wait_stream(cs)
+            self.d2h.wait_stream(cs)
+        self._copy_in(0)
+        for i in range(n_steps):
+            b = i % 2
+            if i + 1 < n_steps:
+                self._copy_in((i + 1) % 2)        # overlaps this step's kernels
+            cs.wait_event(self.ev_in[b])
+            if self.used[b]:
+                cs.wait_event(self.ev_out[b])     # the previous result of this set is home
+            self.hp.use(self.sets[b])
+            self.hp.run_step_kernels(step)
+            self.ev_used[b].record(cs)
+            self.used[b] = True
+            self.d2h.wait_event(self.ev_used[b])
+            with torch.cuda.stream(self.d2h):
+                self.host_out.copy_(self.sets[b]["out"], non_blocking=True)
+            self.ev_out[b].record(self.d2h)
+        if end is not None:
+            cs.wait_stream(self.d2h)
+            cs.wait_stream(self.h2d)
+            end.record(cs)
