@@ -210,7 +210,7 @@ def cpu_oracle_step_time(w, inp, k_cache, v_cache, budget_rows=8, rng_seed=0):
     return est, flops, "; ".join(parts) + " (single-threaded fp64 C, extrapolated per stage)"
 
 
-def measure_projections(J, hp, step, stream, pk, reps=10):
+def measure_projections(J, hp, step, stream, pk, reps=10, cpu_rows=0):
     """The block's projections on the step's active tokens (outside the hot
     path's step, reported beside it): the fused Q/K/V projection that writes
     K/V straight into the cache, and the output projection scattered back to
@@ -250,6 +250,23 @@ def measure_projections(J, hp, step, stream, pk, reps=10):
     code = J.device_error(stream)
     if code:
         raise RuntimeError(f"device error in projections: {J.jano_status_str(code)}")
+    if cpu_rows:
+        # the fp64 CPU oracle on a bounded sample: cpu_rows active rows of the
+        # fused projection, extrapolated to all n_act rows
+        import oracle
+        import synth
+        oracle.build()
+        rows = idx[:cpu_rows].cpu().numpy()
+        xb = synth.bits_of(x[torch.from_numpy(rows).long().to(hp.dev)].cpu())
+        wb = synth.bits_of(w_qkv.cpu())
+        t0 = time.perf_counter()
+        oracle.gather_gemm(xb, wb)
+        dt = (time.perf_counter() - t0) * n_act / cpu_rows
+        fl = res["qkv_project"]["flops"]
+        res["qkv_project"]["cpu_oracle"] = {
+            "TFLOP/s": fl / dt / 1e12, "cores": 1, "kind": "oracle",
+            "sample": f"{cpu_rows} of {n_act} rows x {3 * hd} outputs x k={hd} "
+                      "(single-threaded fp64 C, extrapolated)"}
     return res
 
 
@@ -405,7 +422,8 @@ def run_gpu(args, w, rank, world, local_rank, dist):
 
     next_rows = None
     if not args.no_next:
-        next_rows = measure_projections(J, hp, step, stream, pk)
+        next_rows = measure_projections(J, hp, step, stream, pk,
+                                        cpu_rows=0 if args.no_cpu_baseline or world > 1 else 2)
 
     cfg = workload_config(w)
     cfg.update({"n_active": n_act, "global_batch": world, "parallelism": f"replicas x{world}",
