@@ -7,7 +7,8 @@
 //
 //   out_seg(r)[dst_seg(r)][j] = sum_c x[src(r)][c] * w[j][c]
 //
-// One CTA per 128-row x BN-column output tile, 9 warps:
+// A persistent grid, one CTA per SM, walks the 128-row x BN-column output
+// tiles; 9 warps:
 //   warps 0-3  producers.  The tile's 128 source rows (src(r) = gather[r],
 //            or r) are read once into shared memory.  Per 64-column K block
 //            the A rows are gathered with 16-byte cp.async copies (eight
@@ -19,12 +20,13 @@
 //            (the barrier cannot complete before that thread's copies have
 //            landed) plus an ordinary arrive, so it never waits for its own
 //            copies and runs as far ahead as the ring allows.
-//   warp 4   allocates BN TMEM columns; one lane issues tcgen05.mma
-//            (kind::f16, M=128, N=BN, K=16, both operands K-major from shared
-//            memory, fp32 accumulator in TMEM) and frees ring slots with
-//            tcgen05.commit.
-//   warps 5-8  epilogue: thread = one output row = one TMEM lane; the
-//            accumulator is read 32 columns at a time, rounded to BF16 and
+//   warp 4   allocates 2 x BN TMEM columns (two accumulators); one lane
+//            issues tcgen05.mma (kind::f16, M=128, N=BN, K=16, both operands
+//            K-major from shared memory, fp32 accumulator in TMEM) into the
+//            accumulators in turn and frees ring slots with tcgen05.commit.
+//   warps 5-8  epilogue: thread = one output row = one TMEM lane; a tile's
+//            accumulator (ready while the next tile's MMAs fill the other
+//            one) is read 32 columns at a time, rounded to BF16 and
 //            stored to the row's destination.  The N range may be cut into
 //            segments with their own destination and row map, which is how
 //            the fused Q/K/V projection writes Q to the active rows and K, V
@@ -75,9 +77,11 @@ struct PLayout {
     static constexpr uint32_t kB = BN * PK * 2;                  // 32 KB for BN = 256
     static constexpr uint32_t kStage = kA + kB;
     static constexpr uint32_t kBar = kStages * kStage;
-    static constexpr int bFull = 0, bEmpty = kStages, bAcc = 2 * kStages, kNumBars = 2 * kStages + 1;
-    static constexpr uint32_t kRows = kBar + 8 * kNumBars;       // int32 [PM]
-    static constexpr uint32_t kMisc = kRows + 4 * PM;            // tmem base, abort flag
+    // ring full/empty, accumulator full [2] (MMA commit), accumulator empty
+    // [2] (the 4 epilogue warps), the final drain
+    static constexpr int bFull = 0, bEmpty = kStages, bAccFull = 2 * kStages,
+                         bAccEmpty = bAccFull + 2, bFinal = bAccEmpty + 2, kNumBars = bFinal + 1;
+    static constexpr uint32_t kMisc = kBar + 8 * kNumBars;       // tmem base, abort flag
     static constexpr uint32_t kBytes = kMisc + 16;
     static constexpr uint32_t kAlloc = kBytes + 1024;            // slack for 1 KB alignment
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
@@ -129,6 +133,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1) : "memory");
 }
 
+// Output tile number t of the grouped rasterisation: consecutive tiles walk
+// the column tiles of a group of kGroupM row tiles.
+__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int& m_tile, int& n_tile) {
+    const int per_group = kGroupM * n_tiles;
+    const int group = t / per_group;
+    const int first_m = group * kGroupM;
+    const int gm = min(kGroupM, m_tiles - first_m);
+    m_tile = first_m + (t % per_group) % gm;
+    n_tile = (t % per_group) / gm;
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 projection_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ GemmArgs a) {
@@ -139,18 +154,9 @@ projection_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
     uint8_t* gbase = smem_raw + (base - raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // grouped rasterisation: consecutive CTAs walk the column tiles of a
-    // group of kGroupM row tiles
     const int n_tiles = (a.n + BN - 1) / BN;
     const int m_tiles = (a.m + PM - 1) / PM;
-    const int pid = blockIdx.x;
-    const int per_group = kGroupM * n_tiles;
-    const int group = pid / per_group;
-    const int first_m = group * kGroupM;
-    const int gm = min(kGroupM, m_tiles - first_m);
-    const int m_tile = first_m + (pid % per_group) % gm;
-    const int n_tile = (pid % per_group) / gm;
-    const int m0 = m_tile * PM, n0 = n_tile * BN;
+    const int tiles = n_tiles * m_tiles;
     const int nkb = (a.k + PK - 1) / PK;
 
     PCtl ctl;
@@ -158,7 +164,6 @@ projection_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
     ctl.abort = reinterpret_cast<volatile int*>(gbase + L::kMisc + 4);
     ctl.err = a.err;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kMisc);
-    int* rows = reinterpret_cast<int*>(gbase + L::kRows);
 
     if (threadIdx.x == 0) {
         ptx::prefetch_tmap(&tmB);
@@ -167,28 +172,16 @@ projection_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
             ptx::mbar_init(ctl.bar(L::bFull + s), kProducers + 1);
             ptx::mbar_init(ctl.bar(L::bEmpty + s), 1);
         }
-        ptx::mbar_init(ctl.bar(L::bAcc), 1);
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(ctl.bar(L::bAccFull + b), 1);
+            ptx::mbar_init(ctl.bar(L::bAccEmpty + b), 4);
+        }
+        ptx::mbar_init(ctl.bar(L::bFinal), 1);
         *ctl.abort = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == 0) {
-        // source rows of the tile; rows past m and bad indices become -1
-        // (their copies write zeros)
-        for (int i = lane; i < PM; i += 32) {
-            const int r = m0 + i;
-            int src = -1;
-            if (r < a.m) {
-                src = a.gather ? __ldg(a.gather + r) : r;
-                if (src < 0 || src >= a.n_x) {
-                    raise_error(a.err, JANO_EINDEX);
-                    src = -1;
-                }
-            }
-            rows[i] = src;
-        }
-    }
     if (warp == kMmaWarp) {
-        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), BN);
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), 2 * BN);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
@@ -202,89 +195,120 @@ projection_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
         const int c = t & 7;                          // 16-byte chunk of a 128-byte row
         const int rg = t >> 3;                        // first row (rows rg, rg+16, ...)
         const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(a.x);
-        int src[PM / 16];
-#pragma unroll
-        for (int u = 0; u < PM / 16; ++u) src[u] = rows[rg + 16 * u];
-        int kb = 0;
-        for (; kb < nkb; ++kb) {
-            const int s = kb % kStages;
-            // warp-uniform: lane 0 waits, the warp follows
-            if (!ctl.warp_wait(L::bEmpty + s, ((kb / kStages) & 1) ^ 1)) break;
-            const uint32_t sa = base + s * L::kStage;
-            const uint32_t full = ctl.bar(L::bFull + s);
-            if (t == 0) {
-                ptx::mbar_arrive_expect_tx(full, L::kB);
-                tma_load_2d(sa + L::kA, &tmB, full, kb * PK, n0);
-            }
-            const int col = kb * PK + 8 * c;          // first element of this thread's chunk
-            const uint32_t bytes_k = col < a.k ? 16u : 0u;
+        int q = 0;                                    // stage counter, across tiles
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+            int mt, nt;
+            tile_coords(tile, m_tiles, n_tiles, mt, nt);
+            const int m0 = mt * PM, n0 = nt * BN;
+            // this thread's 8 source rows; rows past m and bad indices copy zeros
+            int src[PM / 16];
 #pragma unroll
             for (int u = 0; u < PM / 16; ++u) {
-                const int i = rg + 16 * u;            // row of the tile
-                const bool live = src[u] >= 0 && bytes_k;
-                const void* g = live ? static_cast<const void*>(xb + (size_t)src[u] * a.k + col) : a.x;
-                cp_async16(sa + i * 128 + ((c ^ (i & 7)) << 4), g, live ? 16u : 0u);
+                const int r = m0 + rg + 16 * u;
+                int sr = -1;
+                if (r < a.m) {
+                    sr = a.gather ? __ldg(a.gather + r) : r;
+                    if (sr < 0 || sr >= a.n_x) {
+                        if (nt == 0) raise_error(a.err, JANO_EINDEX);
+                        sr = -1;
+                    }
+                }
+                src[u] = sr;
             }
-            cp_async_arrive(full);
-            ptx::mbar_arrive(full);
+            for (int kb = 0; kb < nkb; ++kb, ++q) {
+                const int s = q % kStages;
+                // warp-uniform: lane 0 waits, the warp follows
+                if (!ctl.warp_wait(L::bEmpty + s, ((q / kStages) & 1) ^ 1)) { ok = false; break; }
+                const uint32_t sa = base + s * L::kStage;
+                const uint32_t full = ctl.bar(L::bFull + s);
+                if (t == 0) {
+                    ptx::mbar_arrive_expect_tx(full, L::kB);
+                    tma_load_2d(sa + L::kA, &tmB, full, kb * PK, n0);
+                }
+                const int col = kb * PK + 8 * c;      // first element of this thread's chunk
+                const bool in_k = col < a.k;
+#pragma unroll
+                for (int u = 0; u < PM / 16; ++u) {
+                    const int i = rg + 16 * u;        // row of the tile
+                    const bool live = src[u] >= 0 && in_k;
+                    const void* g = live ? static_cast<const void*>(xb + (size_t)src[u] * a.k + col) : a.x;
+                    cp_async16(sa + i * 128 + ((c ^ (i & 7)) << 4), g, live ? 16u : 0u);
+                }
+                cp_async_arrive(full);
+                ptx::mbar_arrive(full);
+            }
         }
         // no copy outlives the CTA (after a timeout some stages are never consumed)
         cp_async_wait_all();
         if (t == 0) {
             // drain: every weight copy this CTA issued lands before its smem is released
-            for (int q = (kb > kStages ? kb - kStages : 0); q < kb; ++q)
-                ptx::mbar_wait(ctl.bar(L::bFull + q % kStages), (q / kStages) & 1, kWaitLimit);
+            for (int r = (q > kStages ? q - kStages : 0); r < q; ++r)
+                ptx::mbar_wait(ctl.bar(L::bFull + r % kStages), (r / kStages) & 1, kWaitLimit);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_bf16(PM, BN, false, false);
+            int q = 0, lt = 0;
             bool ok = true;
-            for (int kb = 0; kb < nkb; ++kb) {
-                const int s = kb % kStages;
-                if (!ctl.wait(L::bFull + s, (kb / kStages) & 1)) { ok = false; break; }
-                fence_proxy_async();
+            for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x, ++lt) {
+                const int b = lt & 1;
+                // the epilogue has read this accumulator's previous tile
+                if (!ctl.wait(L::bAccEmpty + b, ((lt >> 1) & 1) ^ 1)) { ok = false; break; }
                 ptx::tc_fence_after();
-                const uint32_t sa = base + s * L::kStage;
+                const uint32_t acc = tmem + b * BN;
+                for (int kb = 0; kb < nkb; ++kb, ++q) {
+                    const int s = q % kStages;
+                    if (!ctl.wait(L::bFull + s, (q / kStages) & 1)) { ok = false; break; }
+                    fence_proxy_async();
+                    ptx::tc_fence_after();
+                    const uint32_t sa = base + s * L::kStage;
 #pragma unroll
-                for (int kk = 0; kk < PK / 16; ++kk)
-                    ptx::mma_ss(tmem, ptx::smem_desc_sw128(sa + kk * 32, 16, 1024),
-                                ptx::smem_desc_sw128(sa + L::kA + kk * 32, 16, 1024), idesc,
-                                (kb > 0 || kk > 0) ? 1u : 0u);
-                ptx::mma_commit(ctl.bar(L::bEmpty + s));
+                    for (int kk = 0; kk < PK / 16; ++kk)
+                        ptx::mma_ss(acc, ptx::smem_desc_sw128(sa + kk * 32, 16, 1024),
+                                    ptx::smem_desc_sw128(sa + L::kA + kk * 32, 16, 1024), idesc,
+                                    (kb > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_commit(ctl.bar(L::bEmpty + s));
+                }
+                if (ok) ptx::mma_commit(ctl.bar(L::bAccFull + b));
             }
-            // the accumulator is complete (or, after a timeout, every MMA has
-            // drained); TMEM is released only after that
-            (void)ok;
-            ptx::mma_commit(ctl.bar(L::bAcc));
-            ptx::mbar_wait(ctl.bar(L::bAcc), 0, kWaitLimit);
+            // every MMA of this CTA completes before TMEM is released
+            ptx::mma_commit(ctl.bar(L::bFinal));
+            ptx::mbar_wait(ctl.bar(L::bFinal), 0, kWaitLimit);
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;                       // TMEM lane quarter of this warp
-        const int row = q * 32 + lane;
-        const int r = m0 + row;
-        const int seg_i = n0 / a.seg_w;
-        const Seg& sg = a.seg[seg_i];
-        const int col0 = n0 - seg_i * a.seg_w;        // first column of the tile in its segment
-        int dst_row = -1;
-        if (r < a.m) {
-            dst_row = sg.rowmap ? __ldg(sg.rowmap + r) : r;
-            if (dst_row < 0 || dst_row >= sg.n_rows) {
-                raise_error(a.err, JANO_EINDEX);
-                dst_row = -1;
-            }
-        }
-        if (ctl.warp_wait(L::bAcc, 0) && !*ctl.abort) {
+        const int qd = warp & 3;                      // TMEM lane quarter of this warp
+        const int row = qd * 32 + lane;
+        int lt = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++lt) {
+            const int b = lt & 1;
+            if (!ctl.warp_wait(L::bAccFull + b, (lt >> 1) & 1) || *ctl.abort) break;
             ptx::tc_fence_after();
-            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16);
+            int mt, nt;
+            tile_coords(tile, m_tiles, n_tiles, mt, nt);
+            const int m0 = mt * PM, n0 = nt * BN;
+            const int r = m0 + row;
+            const int seg_i = n0 / a.seg_w;
+            const Seg& sg = a.seg[seg_i];
+            const int col0 = n0 - seg_i * a.seg_w;    // first column of the tile in its segment
+            int dst_row = -1;
+            if (r < a.m) {
+                dst_row = sg.rowmap ? __ldg(sg.rowmap + r) : r;
+                if (dst_row < 0 || dst_row >= sg.n_rows) {
+                    raise_error(a.err, JANO_EINDEX);
+                    dst_row = -1;
+                }
+            }
+            const uint32_t taddr = tmem + b * BN + ((uint32_t)(qd * 32) << 16);
             __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(sg.dst) +
                                   (size_t)(dst_row < 0 ? 0 : dst_row) * sg.ld + col0;
             const int cols = min(BN, a.seg_w - col0);  // columns of this tile inside the segment
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int cc = 0; cc < BN / 32; ++cc) {
                 uint32_t v[32];
-                ptx::tmem_ld32(taddr + 32 * c, v);
+                ptx::tmem_ld32(taddr + 32 * cc, v);
                 ptx::tmem_wait_ld();
                 uint32_t pk[16];
 #pragma unroll
@@ -293,18 +317,22 @@ projection_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
                 if (dst_row >= 0) {
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
-                        if (32 * c + 8 * u < cols)
-                            *reinterpret_cast<uint4*>(orow + 32 * c + 8 * u) =
+                        if (32 * cc + 8 * u < cols)
+                            *reinterpret_cast<uint4*>(orow + 32 * cc + 8 * u) =
                                 make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
                 }
             }
+            // this accumulator may take the next tile
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ctl.bar(L::bAccEmpty + b));
         }
     }
 
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, BN);
+    if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, 2 * BN);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -348,7 +376,10 @@ cudaError_t launch_bn(const void* w, const GemmArgs& a, cudaStream_t st) {
         if (dev < 64) done_mask |= 1ull << dev;
     }
     const int tiles = ((a.m + PM - 1) / PM) * ((a.n + BN - 1) / BN);
-    projection_kernel<BN><<<tiles, kThreads, L::kAlloc, st>>>(mB, a);
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = tiles < sms ? tiles : sms;      // persistent: one CTA per SM
+    projection_kernel<BN><<<grid, kThreads, L::kAlloc, st>>>(mB, a);
     return cudaGetLastError();
 }
 
