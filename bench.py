@@ -169,11 +169,20 @@ def traffic_for(kernel_src_rel):
 
 
 # ------------------------------------------------------------------ CPU oracle
-def cpu_oracle_step_time(w, inp, k_cache, v_cache, budget_rows=8, rng_seed=0):
-    """Time the oracle stage by stage on a bounded sample, extrapolate each
-    stage to the full workload; returns (seconds per full step, sample text)."""
-    import oracle
+def oracle_inputs(inp, k_cache, v_cache, n_act):
+    """BF16 bit arrays of the step's inputs for the CPU oracle (made once)."""
     import synth
+    return {"kb": synth.bits_of(k_cache), "vb": synth.bits_of(v_cache),
+            "qb": synth.bits_of(inp["q_act"][:n_act]), "ka": synth.bits_of(inp["k_act"]),
+            "va": synth.bits_of(inp["v_act"])}
+
+
+def cpu_oracle_step_time(w, inp, bits, budget_rows=8, rng_seed=0):
+    """Time the oracle stage by stage on a bounded sample, extrapolate each
+    stage to the full workload; returns (seconds per full step, FLOPs, sample
+    text).  `bits` holds the BF16 bit arrays of oracle_inputs (the scatter
+    writes into its caches in place)."""
+    import oracle
     oracle.build()
     N, H, d = w.n_tokens, w.heads, w.d
     lat = inp["lat"].numpy()
@@ -188,23 +197,22 @@ def cpu_oracle_step_time(w, inp, k_cache, v_cache, budget_rows=8, rng_seed=0):
     # a2 + a3 in full
     t = time.perf_counter()
     lv = oracle.classify(field, w.frac_active, w.frac_static)
-    pf, ph, pw = w.patch
     off, idx, _ = oracle.build_schedule(lv, (w.F, w.H, w.W), w.patch, w.patch, w.T, w.warmup,
                                         w.cooldown, w.period_moderate, w.period_static)
     est += time.perf_counter() - t; parts.append("classify+schedule full")
     n_act = int(off[w.warmup + 1] - off[w.warmup])
     sel = idx[off[w.warmup]:off[w.warmup + 1]]
-    # a4 on 256 rows
+    # a4 on 256 rows, in place
     m = min(256, n_act)
-    kb, vb = synth.bits_of(k_cache), synth.bits_of(v_cache)
-    ka, va = synth.bits_of(inp["k_act"][:m]), synth.bits_of(inp["v_act"][:m])
-    t = time.perf_counter(); oracle.kv_scatter(ka, va, sel[:m], kb, vb); dt = time.perf_counter() - t
+    t = time.perf_counter()
+    oracle.kv_scatter(bits["ka"][:m], bits["va"][:m], sel[:m], bits["kb"], bits["vb"], inplace=True)
+    dt = time.perf_counter() - t
     est += dt * n_act / m; parts.append(f"scatter {m} rows")
     # a5 on budget_rows rows x all heads x all keys
     g = np.random.default_rng(rng_seed)
     rows = np.sort(g.choice(n_act, size=min(budget_rows, n_act), replace=False)).astype(np.int32)
-    qb = synth.bits_of(inp["q_act"][:n_act])
-    t = time.perf_counter(); oracle.active_attention(qb, kb, vb, rows=rows); dt = time.perf_counter() - t
+    t = time.perf_counter(); oracle.active_attention(bits["qb"], bits["kb"], bits["vb"], rows=rows)
+    dt = time.perf_counter() - t
     est += dt * n_act / rows.size; parts.append(f"attention {rows.size} rows x {H} heads x {N} keys")
     flops = 4.0 * n_act * N * d * H
     return est, flops, "; ".join(parts) + " (single-threaded fp64 C, extrapolated per stage)"
@@ -274,13 +282,16 @@ def run_reference(args, w, rank, world):
     if rank != 0:
         return 0
     inp, k_cache, v_cache, n_cap = make_inputs(w)
+    bits = oracle_inputs(inp, k_cache, v_cache, n_cap)
+    # attention rows per step: the bounded sample shrinks with the step count
+    # so that the whole run stays within a few minutes (about 2.3 s per row)
+    rows = args.ref_rows if args.ref_rows > 0 else max(1, min(8, 60 // max(1, args.steps + args.warmup)))
     times = []
     flops = None
     sample = ""
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        est, flops, sample = cpu_oracle_step_time(w, inp, k_cache, v_cache,
-                                                  budget_rows=args.ref_rows, rng_seed=i)
+        est, flops, sample = cpu_oracle_step_time(w, inp, bits, budget_rows=rows, rng_seed=i)
         if i >= args.warmup:
             times.append(est)
         log(f"reference step {i}: estimated full step {est:.1f} s (wall {time.perf_counter()-t0:.1f} s)")
@@ -416,7 +427,8 @@ def run_gpu(args, w, rank, world, local_rank, dist):
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         t0 = time.perf_counter()
-        est, fl, sample = cpu_oracle_step_time(w, inp, k_cache, v_cache, budget_rows=args.ref_rows)
+        bits = oracle_inputs(inp, k_cache, v_cache, n_cap)
+        est, fl, sample = cpu_oracle_step_time(w, inp, bits, budget_rows=args.ref_rows if args.ref_rows > 0 else 8)
         cpu = {"value": fl / est / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
                "sample": sample, "wall_s": time.perf_counter() - t0}
 
@@ -451,7 +463,9 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--ref-rows", type=int, default=8)
+    ap.add_argument("--ref-rows", type=int, default=0,
+                    help="attention rows per oracle sample (0: 8 for the GPU arm's baseline, "
+                         "sized from --steps/--warmup for --impl reference)")
     ap.add_argument("--no-next", action="store_true",
                     help="skip the projections measured beside the step")
     args = ap.parse_args()

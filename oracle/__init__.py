@@ -135,13 +135,19 @@ def build_schedule(block_levels, dims, block, patch, T, warmup, cooldown,
     return offsets, idx[: offsets[T]].copy(), tl
 
 
-def kv_scatter(k_act, v_act, idx, k_cache, v_cache):
-    """In-place on copies: returns the updated (k_cache, v_cache) uint16 arrays."""
+def kv_scatter(k_act, v_act, idx, k_cache, v_cache, inplace=False):
+    """Returns the updated (k_cache, v_cache) uint16 arrays: copies of the
+    inputs, or (inplace=True, C-contiguous uint16 caches) the caches themselves."""
     k_act = np.ascontiguousarray(k_act, dtype=np.uint16)
     v_act = np.ascontiguousarray(v_act, dtype=np.uint16)
     idx = np.ascontiguousarray(idx, dtype=np.int32)
-    kc = np.array(k_cache, dtype=np.uint16, copy=True, order="C")
-    vc = np.array(v_cache, dtype=np.uint16, copy=True, order="C")
+    if inplace:
+        assert k_cache.dtype == np.uint16 and k_cache.flags.c_contiguous
+        assert v_cache.dtype == np.uint16 and v_cache.flags.c_contiguous
+        kc, vc = k_cache, v_cache
+    else:
+        kc = np.array(k_cache, dtype=np.uint16, copy=True, order="C")
+        vc = np.array(v_cache, dtype=np.uint16, copy=True, order="C")
     n_tokens = kc.shape[0]
     row = int(np.prod(kc.shape[1:]))
     _check("oracle_kv_scatter", _load().oracle_kv_scatter(
