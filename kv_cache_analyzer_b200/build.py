@@ -38,7 +38,8 @@ def _headers():
 def build(force: bool = False, debug: bool = False, verbose: bool = False,
           out: str | None = None, defines: tuple = ()) -> str:
     """Compile and link; `out`/`defines` build a variant (own object dir)."""
-    lib_path = out or LIB
+    lib_path = os.path.abspath(out or LIB)
+    os.makedirs(os.path.dirname(lib_path), exist_ok=True)
     obj_dir = OBJ if not (out or defines) else os.path.join(
         ROOT, "_build", "variant_" + "_".join(d.replace("=", "-") for d in defines))
     os.makedirs(obj_dir, exist_ok=True)

@@ -321,6 +321,11 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
             for (int n = 0; n < 2 * nt; ++n) {
                 const int s = n % kSlots;
                 if (!ctl.wait(L::bEmpty + s, ((n / kSlots) & 1) ^ 1)) break;
+#ifdef JANO_INJECT_DROP_LOAD
+                // failure-path test builds only: this copy is never issued, so
+                // the MMA's bounded wait for it runs out (JANO_ETIMEOUT)
+                if (n == JANO_INJECT_DROP_LOAD) continue;
+#endif
                 ptx::mbar_arrive_expect_tx(ctl.bar(L::bFull + s), L::kTile);
                 const CUtensorMap* tm = (n & 1) ? &tmV : &tmK;
                 for (int p = 0; p < L::kPanels; ++p)
