@@ -1,0 +1,94 @@
+"""The step sharded over ranks (frame slabs for the analyzer, head ranges for
+scatter and attention), emulated on one GPU: the ranks' kernels run one
+after another, each on its own buffers, and the all-gather of block scores
+is a concatenation.  Every rank's scores, schedule, cache heads and output
+heads must equal, bit for bit, the unsharded step's.  No rank waits on
+another inside a kernel, so running them in sequence is exact emulation."""
+import os
+import sys
+
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _geoms(J, w):
+    return (J.Geometry(w.F, w.H, w.W, w.block, w.patch), J.Geometry(w.F, w.H, w.W, w.patch, w.patch),
+            J.Schedule(w.T, w.warmup, w.cooldown, w.period_moderate, w.period_static))
+
+
+def _bits(t):
+    return t.contiguous().view(torch.int16 if t.dtype == torch.bfloat16 else torch.int32).cpu()
+
+
+@pytest.mark.parametrize("name,world", [("tiny", 2), ("small", 2), ("small", 3), ("large", 8)])
+def test_sharded_step_equals_unsharded(name, world):
+    import bench
+    import synth
+    import kv_cache_analyzer_b200 as J
+    from kv_cache_analyzer_b200.pipeline import HotPath
+    from kv_cache_analyzer_b200.sharding import ShardedHotPath
+    w = synth.WORKLOADS[name]
+    inp, k_cache, v_cache, n_cap = bench.make_inputs(w)
+    lg, tg, sc = _geoms(J, w)
+    stream = torch.cuda.Stream()
+    step = w.warmup
+
+    ref = HotPath(K=w.K, C=w.C, latent_geom=lg, token_geom=tg, heads=w.heads, d=w.d,
+                  frac_active=w.frac_active, frac_static=w.frac_static, sched=sc, stream=stream)
+    ref.set_activations(n_cap)
+    with torch.cuda.stream(stream):
+        ref.lat.copy_(inp["lat"]); ref.field.copy_(inp["field"])
+        ref.q_act.copy_(inp["q_act"]); ref.k_act.copy_(inp["k_act"]); ref.v_act.copy_(inp["v_act"])
+        ref.k_cache.copy_(k_cache); ref.v_cache.copy_(v_cache)
+    stream.synchronize()
+    ref.plan()
+    ref.run_step_kernels(step)
+    stream.synchronize()
+    assert J.device_error() == 0
+
+    shards = []
+    for r in range(world):
+        sh = ShardedHotPath(rank=r, world=world, K=w.K, C=w.C, latent_geom=lg, token_geom=tg,
+                            heads=w.heads, d=w.d, frac_active=w.frac_active,
+                            frac_static=w.frac_static, sched=sc, stream=stream)
+        sh.set_activations(n_cap)
+        sh.load_latent(inp["lat"])
+        with torch.cuda.stream(stream):
+            sh.field.copy_(inp["field"])
+            for k in ("q_act", "k_act", "v_act"):
+                getattr(sh, k).copy_(sh.head_slice(inp[k]))
+            sh.k_cache.copy_(sh.head_slice(k_cache)); sh.v_cache.copy_(sh.head_slice(v_cache))
+        shards.append(sh)
+    assert sum(sh.heads for sh in shards) == w.heads
+    assert sum(sh.counts[sh.rank] for sh in shards) == lg.n_blocks
+    # a1 on every rank, then the gather, then a2..a5 on every rank
+    for sh in shards:
+        sh.run_local_scores()
+    with torch.cuda.stream(stream):
+        full = torch.cat([sh.local_scores() for sh in shards])
+        for sh in shards:
+            sh.scores.copy_(full)
+    for sh in shards:
+        sh.run_after_gather()
+    stream.synchronize()
+    for sh in shards:
+        sh.host_offsets = sh.offsets.cpu().tolist()
+        sh.run_head_kernels(step)
+    stream.synchronize()
+    assert J.device_error() == 0
+
+    s_ref = _bits(ref.scores)
+    off_ref = ref.offsets.cpu()
+    n_due = int(off_ref[-1])
+    idx_ref = ref.idx[:n_due].cpu()
+    for sh in shards:
+        assert torch.equal(_bits(sh.scores), s_ref), f"rank {sh.rank} scores"
+        assert torch.equal(sh.offsets.cpu(), off_ref)
+        assert torch.equal(sh.idx[:n_due].cpu(), idx_ref)
+        for mine, theirs in ((sh.k_cache, ref.k_cache), (sh.v_cache, ref.v_cache), (sh.out, ref.out)):
+            assert torch.equal(_bits(mine), _bits(sh.head_slice(theirs))), f"rank {sh.rank} heads"
