@@ -17,7 +17,8 @@ has no data-path exchange, so N GPUs process N problems ("weak" scaling).
 Beside the step (not in its value) the line reports ``next_rows``: the
 block's projections on the step's active tokens -- the fused Q/K/V projection
 writing K/V straight into the cache and the output projection scattered back
-to the token rows -- with their TFLOP/s.
+to the token rows -- with their TFLOP/s, and the FFT baseline score with
+the analyzer timed under the same conditions (HBM GB/s).
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead, on
 a bounded sample of the same workload, extrapolated stage by stage to the
@@ -278,6 +279,48 @@ def measure_projections(J, hp, step, stream, pk, reps=10, cpu_rows=0):
     return res
 
 
+def measure_fft_score(J, hp, stream, pk, reps=10, cutoff=1):
+    """The FFT baseline score (outside the step, reported beside it) against
+    the analyzer under the same conditions: each launch alone, L2 flushed
+    before it (a 256 MB write), on the last warm-up snapshot x_K.  The FFT
+    score reads one snapshot; the analyzer reads all K+1."""
+    import torch
+    K, C = hp.K, hp.C
+    x = hp.lat[K]
+    out = torch.empty_like(hp.scores)
+    geom = hp.lg.c()
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=hp.dev)
+    snap_bytes = float(x.numel()) * 4 + out.numel() * 4
+    lat_bytes = float(hp.lat.numel()) * 4 + out.numel() * 4
+    ops = {
+        "fft_score": (lambda: J.jano_fft_scores(x, C, geom, cutoff, out, stream), snap_bytes),
+        "block_scores_same_conditions": (lambda: J.jano_block_scores(hp.lat, K, C, geom, hp.w_t, hp.w_s,
+                                                                     out, stream), lat_bytes),
+    }
+    res = {}
+    for name, (fn, nbytes) in ops.items():
+        for _ in range(3):
+            fn()
+        ms = []
+        for _ in range(reps):
+            with torch.cuda.stream(stream):
+                flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            stream.synchronize()
+            ms.append(a.elapsed_time(b))
+        m = sorted(ms)[reps // 2]
+        gbs = nbytes / (m * 1e-3) / 1e9
+        res[name] = {"ms": m, "GB/s": gbs, "frac_of_hbm": gbs / pk["hbm_gbs"], "algorithmic_bytes": nbytes}
+    res["fft_score"]["cutoff"] = cutoff
+    code = J.device_error(stream)
+    if code:
+        raise RuntimeError(f"device error in the FFT score: {J.jano_status_str(code)}")
+    return res
+
+
 def run_reference(args, w, rank, world):
     if rank != 0:
         return 0
@@ -436,6 +479,7 @@ def run_gpu(args, w, rank, world, local_rank, dist):
     if not args.no_next:
         next_rows = measure_projections(J, hp, step, stream, pk,
                                         cpu_rows=0 if args.no_cpu_baseline or world > 1 else 2)
+        next_rows.update(measure_fft_score(J, hp, stream, pk))
 
     cfg = workload_config(w)
     cfg.update({"n_active": n_act, "global_batch": world, "parallelism": f"replicas x{world}",

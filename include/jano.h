@@ -313,6 +313,36 @@ JANO_API jano_status jano_qkv_project(const void *x, int n_tokens, const int32_t
  * ---------------------------------------------------------------------- */
 JANO_API jano_status jano_random_scores(int n_blocks, uint64_t seed, float *scores, void *stream);
 
+/* ------------------------------------------------------------------------
+ * jano_fft_scores -- frequency-domain block complexity, the FFT baseline
+ * the analyzer is compared with.  Pages: zh technical summary 1 (an FFT
+ * complexity analysis cannot tell the patterns apart in the early,
+ * noise-dominated steps) and 2.1 (FFT on the early latent: median
+ * prediction accuracy 0.13-0.25 against the analyzer's 0.73); fr technical
+ * summary 2.A.  The pages give no formula; this is its plainest form, on one
+ * latent snapshot x (normally the last warm-up step's, x_K):
+ *
+ *   S_b = 1/C sum_c 1/n_b^2 sum_{u in U_hi} |X_{c,b}(u)|^2
+ *
+ * X_{c,b} is the 3-D DFT of block b of channel c over the block's own
+ * m_f x m_h x m_w elements (edge blocks are smaller, n_b = m_f m_h m_w), and
+ * U_hi holds the frequencies u whose folded index min(u_a, m_a - u_a)
+ * reaches `cutoff` on at least one axis a.  By Parseval's theorem cutoff 0
+ * gives the block's mean square and cutoff 1 its variance (all but the DC
+ * bin); a cutoff above every folded index gives 0.  Blocks are ordered as in
+ * jano_block_scores, so jano_classify takes these scores unchanged.
+ *
+ * x       device fp32 [C][F][H][W], one snapshot (4-byte aligned).
+ * g       block geometry (bf, bh, bw); the patch fields are not read.
+ *         bf * bh * bw <= 256 (JANO_EUNSUPPORTED beyond).
+ * cutoff  >= 0.
+ * scores  device fp32 [n_blocks].
+ * Errors: JANO_EINVAL (NULL pointer, C < 1, cutoff < 0, bad geometry),
+ * JANO_EUNSUPPORTED, JANO_ECUDA.  Deterministic: fixed summation order.
+ * ---------------------------------------------------------------------- */
+JANO_API jano_status jano_fft_scores(const float *x, int C, const jano_geom *g, int cutoff,
+                                     float *scores, void *stream);
+
 /* Synchronises `stream`, returns the first device-side error recorded on the
  * current device since the last call (JANO_OK if none) and clears it. */
 JANO_API jano_status jano_get_device_error(void *stream);

@@ -38,7 +38,7 @@ STATUS_NAMES = {0: "JANO_OK", 1: "JANO_EINVAL", 2: "JANO_ESHAPE", 3: "JANO_EALIG
                 7: "JANO_ETIMEOUT", 8: "JANO_ECUDA"}
 EXPORTS = ("jano_block_scores", "jano_block_scores_literal", "jano_classify", "jano_build_schedule_workspace_bytes",
            "jano_build_schedule", "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention",
-           "jano_gather_gemm", "jano_qkv_project", "jano_random_scores",
+           "jano_gather_gemm", "jano_qkv_project", "jano_random_scores", "jano_fft_scores",
            "jano_get_device_error", "jano_status_str", "jano_version")
 
 
@@ -81,13 +81,15 @@ def lib() -> C.CDLL:
         L.jano_gather_gemm.argtypes = [P, i, P, i, P, i, i, P, P, i, P]
         L.jano_qkv_project.argtypes = [P, i, P, i, P, i, i, P, P, P, P]
         L.jano_random_scores.argtypes = [i, C.c_uint64, P, P]
+        L.jano_fft_scores.argtypes = [P, i, G, i, P, P]
         L.jano_get_device_error.argtypes = [P]
         L.jano_status_str.argtypes = [i]
         L.jano_status_str.restype = C.c_char_p
         L.jano_version.argtypes = []
         for fn in ("jano_block_scores", "jano_block_scores_literal", "jano_classify", "jano_build_schedule",
                    "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention", "jano_get_device_error",
-                   "jano_gather_gemm", "jano_qkv_project", "jano_random_scores", "jano_version"):
+                   "jano_gather_gemm", "jano_qkv_project", "jano_random_scores", "jano_fft_scores",
+                   "jano_version"):
             getattr(L, fn).restype = C.c_int
         _lib = L
     return _lib
@@ -195,6 +197,12 @@ def jano_qkv_project(x, n_tokens, idx, n_act, w_qkv, hd, k, q_act, k_cache, v_ca
 def jano_random_scores(n_blocks, seed, scores, stream=None):
     _check("jano_random_scores", lib().jano_random_scores(
         n_blocks, C.c_uint64(seed), _dev(scores, "scores", torch.float32), _stream(stream)))
+
+
+def jano_fft_scores(x, C_, geom, cutoff, scores, stream=None):
+    _check("jano_fft_scores", lib().jano_fft_scores(
+        _dev(x, "x", torch.float32), C_, geom, cutoff, _dev(scores, "scores", torch.float32),
+        _stream(stream)))
 
 
 def jano_get_device_error(stream=None) -> int:
@@ -328,6 +336,15 @@ def random_scores(n_blocks: int, seed: int, out=None, stream=None) -> torch.Tens
     if out is None:
         out = torch.empty(n_blocks, dtype=torch.float32, device="cuda")
     jano_random_scores(n_blocks, seed, out, stream)
+    return out
+
+
+def fft_scores(x: torch.Tensor, geom: Geometry, cutoff: int = 1, out=None, stream=None) -> torch.Tensor:
+    """High-band spectral energy per block of one snapshot x [C][F][H][W]
+    (the FFT baseline score)."""
+    if out is None:
+        out = torch.empty(geom.n_blocks, dtype=torch.float32, device=x.device)
+    jano_fft_scores(x, x.shape[0], geom.c(), cutoff, out, stream)
     return out
 
 

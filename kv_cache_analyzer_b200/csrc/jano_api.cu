@@ -200,6 +200,16 @@ jano_status jano_random_scores(int n_blocks, uint64_t seed, float* scores, void*
     return from_cuda(launch_random_scores(n_blocks, seed, scores, static_cast<cudaStream_t>(stream)));
 }
 
+jano_status jano_fft_scores(const float* x, int C, const jano_geom* g, int cutoff, float* scores,
+                            void* stream) {
+    if (!x || !scores || C < 1 || cutoff < 0) return JANO_EINVAL;
+    const jano_status gs = check_geom(g, false);
+    if (gs != JANO_OK) return gs;
+    if ((long long)C * g->F * g->H * g->W > (1ll << 40)) return JANO_EUNSUPPORTED;
+    if (!fft_scores_supported(*g)) return JANO_EUNSUPPORTED;
+    return from_cuda(launch_fft_scores(x, C, *g, cutoff, scores, static_cast<cudaStream_t>(stream)));
+}
+
 jano_status jano_get_device_error(void* stream) {
     int* err = device_error_word();
     if (!err) return JANO_ECUDA;

@@ -28,6 +28,9 @@ int* device_error_word();   // address of this device's error word (host)
 cudaError_t launch_block_scores(const float* lat, int K, int C, const jano_geom& g,
                                 float w_t, float w_s, bool literal, float* scores, int* err,
                                 cudaStream_t st);
+bool fft_scores_supported(const jano_geom& g);
+cudaError_t launch_fft_scores(const float* x, int C, const jano_geom& g, int cutoff, float* scores,
+                              cudaStream_t st);
 cudaError_t launch_classify(const float* scores, int n, long long k_static,
                             long long k_active, uint8_t* levels, int* err,
                             cudaStream_t st);

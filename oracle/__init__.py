@@ -61,9 +61,10 @@ def _load():
         lib.oracle_splitmix64.argtypes = [C.c_uint64, i, P]
         lib.oracle_splitmix64.restype = None
         lib.oracle_random_scores.argtypes = [i, C.c_uint64, P]
+        lib.oracle_fft_scores.argtypes = [P, i, i, i, i, i, i, i, i, P]
         for fn in ("oracle_block_scores", "oracle_block_scores_literal", "oracle_level_counts", "oracle_classify",
                    "oracle_build_schedule", "oracle_kv_scatter", "oracle_active_attention",
-                   "oracle_gather_gemm", "oracle_random_scores"):
+                   "oracle_gather_gemm", "oracle_random_scores", "oracle_fft_scores"):
             getattr(lib, fn).restype = C.c_int
         _lib = lib
     return _lib
@@ -192,6 +193,19 @@ def splitmix64(seed, n):
     """The first n outputs of splitmix64 seeded with `seed` (uint64)."""
     out = np.empty(n, dtype=np.uint64)
     _load().oracle_splitmix64(C.c_uint64(seed), n, _ptr(out))
+    return out
+
+
+def fft_scores(x, block, cutoff):
+    """High-band spectral energy per block of one snapshot.
+    x fp32 [C][F][H][W] -> fp64 scores [nBf*nBh*nBw]."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    Cc, F, H, W = x.shape
+    bf, bh, bw = block
+    nB = (-(-F // bf)) * (-(-H // bh)) * (-(-W // bw))
+    out = np.empty(nB, dtype=np.float64)
+    _check("oracle_fft_scores", _load().oracle_fft_scores(_ptr(x), Cc, F, H, W, bf, bh, bw, cutoff,
+                                                          _ptr(out)))
     return out
 
 

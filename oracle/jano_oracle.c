@@ -452,3 +452,69 @@ int oracle_block_scores_literal(const float *lat, int K, int C, int F, int H, in
     free(cnt);
     return OR_OK;
 }
+
+/*
+ * Frequency-domain block complexity, the FFT baseline the analyzer is
+ * compared with (zh page, technical summary 1 and 2.1: an FFT taken on the
+ * early latent predicts convergence poorly; fr page 2.A).  The pages give
+ * no formula; the reading is the energy of the high band of each block's
+ * 3-D discrete Fourier transform, on one snapshot x[c][f][h][w]:
+ *
+ *   X_{c,b}(u) = sum over the block's own elements (f, h, w) of
+ *                x[c][f0+f][h0+h][w0+w] exp(-2 pi i (u_f f/m_f + u_h h/m_h + u_w w/m_w))
+ *   S_b = 1/C sum_c 1/n_b^2 sum_{u : max_a min(u_a, m_a - u_a) >= cutoff} |X_{c,b}(u)|^2
+ *
+ * m_a the block's extent along axis a inside the tensor (edge blocks are
+ * smaller), n_b = m_f m_h m_w.  The DFT is taken by this definition, one
+ * frequency at a time, in fp64 with the C library's cos and sin.
+ */
+static int or_fold(int u, int m) { return u < m - u ? u : m - u; }
+
+int oracle_fft_scores(const float *x, int C, int F, int H, int W, int bf, int bh, int bw,
+                      int cutoff, double *scores)
+{
+    if (!x || !scores || C < 1 || F < 1 || H < 1 || W < 1 || bf < 1 || bh < 1 || bw < 1 ||
+        cutoff < 0)
+        return OR_EINVAL;
+    const int nBf = ceil_div(F, bf), nBh = ceil_div(H, bh), nBw = ceil_div(W, bw);
+    const size_t plane = (size_t)H * W;
+    const size_t vol = (size_t)F * plane;
+    const double two_pi = 2.0 * acos(-1.0);
+    for (int fb = 0; fb < nBf; ++fb)
+        for (int hb = 0; hb < nBh; ++hb)
+            for (int wb = 0; wb < nBw; ++wb) {
+                const int f0 = fb * bf, h0 = hb * bh, w0 = wb * bw;
+                const int mf = F - f0 < bf ? F - f0 : bf;
+                const int mh = H - h0 < bh ? H - h0 : bh;
+                const int mw = W - w0 < bw ? W - w0 : bw;
+                const double n = (double)mf * mh * mw;
+                double total = 0.0;
+                for (int c = 0; c < C; ++c) {
+                    double e = 0.0;
+                    for (int uf = 0; uf < mf; ++uf)
+                        for (int uh = 0; uh < mh; ++uh)
+                            for (int uw = 0; uw < mw; ++uw) {
+                                int k = or_fold(uf, mf);
+                                if (or_fold(uh, mh) > k) k = or_fold(uh, mh);
+                                if (or_fold(uw, mw) > k) k = or_fold(uw, mw);
+                                if (k < cutoff) continue;
+                                double re = 0.0, im = 0.0;
+                                for (int f = 0; f < mf; ++f)
+                                    for (int h = 0; h < mh; ++h)
+                                        for (int w = 0; w < mw; ++w) {
+                                            const double v = x[(size_t)c * vol + (size_t)(f0 + f) * plane +
+                                                               (size_t)(h0 + h) * W + (w0 + w)];
+                                            const double ph = two_pi * ((double)uf * f / mf +
+                                                                        (double)uh * h / mh +
+                                                                        (double)uw * w / mw);
+                                            re += v * cos(ph);
+                                            im -= v * sin(ph);
+                                        }
+                                e += re * re + im * im;
+                            }
+                    total += e / (n * n);
+                }
+                scores[((size_t)fb * nBh + hb) * nBw + wb] = total / C;
+            }
+    return OR_OK;
+}

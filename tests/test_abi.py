@@ -93,6 +93,14 @@ def test_host_validation_rejects_before_any_launch(jl):
     assert L.jano_gather_gemm(nil, 8, nil, 0, nil, 64, 64, nil, nil, 64, nil) == 0
     assert L.jano_qkv_project(fake, 100, fake, 10, fake, 96, 64, fake, fake, fake, nil) == 4
     assert L.jano_qkv_project(nil, 100, nil, 0, nil, 128, 64, nil, nil, nil, nil) == 0
+    # FFT score: negative cutoff, no channels, NULL snapshot, a block of more
+    # than 256 elements
+    g4 = jl.Geometry(4, 32, 32, (1, 4, 4), (1, 2, 2)).c()
+    assert L.jano_fft_scores(fake, 16, C.byref(g4), -1, fake, nil) == 1
+    assert L.jano_fft_scores(fake, 0, C.byref(g4), 1, fake, nil) == 1
+    assert L.jano_fft_scores(nil, 16, C.byref(g4), 1, fake, nil) == 1
+    g5 = jl.Geometry(4, 32, 32, (4, 8, 16), (1, 2, 2)).c()
+    assert L.jano_fft_scores(fake, 16, C.byref(g5), 1, fake, nil) == 4
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch, jl):

@@ -1,7 +1,8 @@
 """GPU parity of the method variants next to the hot path: the random-masking
 ablation's scores and level maps (bit-exact: counter-based generator and
-integer ranks) and the Static refresh period of the pages' example (every
-5th step), through the C ABI."""
+integer ranks), the Static refresh period of the pages' example (every
+5th step), the literal score reading and the FFT baseline score, through the
+C ABI."""
 import numpy as np
 import pytest
 import torch
@@ -85,3 +86,69 @@ def test_literal_scores_edge_geometries(J, shape, block):
     ref = oracle.block_scores_literal(lat, block)
     bound = 1e-5 * np.abs(ref) + 2.0 ** -19 * float(np.abs(lat).max())
     assert np.all(np.abs(got - ref) <= bound)
+
+
+# ---------------------------------------------------------------- FFT baseline score
+def _fft_bound(x, block, ref):
+    """fp32 against fp64, from the arithmetic: each DFT bin is a sum of n_b
+    terms (twiddles exact or correctly rounded), so its error is at most
+    about (n_b + 2) 2^-24 sum|x|; squared, summed over at most n_b bins and
+    divided by n_b^2 that is 2 (n_b + 2) 2^-24 n_b M_b with M_b the channel
+    mean of (mean |x| over the block)^2.  Bound: 2^-16 |ref| + that."""
+    Cc, F, H, W = x.shape
+    bf, bh, bw = block
+    ax = np.abs(x.astype(np.float64))
+    out = np.empty_like(ref)
+    b = 0
+    for f0 in range(0, F, bf):
+        for h0 in range(0, H, bh):
+            for w0 in range(0, W, bw):
+                blk = ax[:, f0:f0 + bf, h0:h0 + bh, w0:w0 + bw]
+                n = blk[0].size
+                M = np.mean(blk.reshape(Cc, -1).mean(axis=1) ** 2)
+                out[b] = 2.0 ** -16 * abs(ref[b]) + 2 * (n + 2) * 2.0 ** -24 * n * M
+                b += 1
+    return out
+
+
+@pytest.mark.parametrize("name", ["tiny", "image", "small", "large"])
+@pytest.mark.parametrize("cutoff", [1, 2])
+def test_fft_scores_match_oracle(J, name, cutoff):
+    import synth
+    from workloads import latent
+    w = synth.WORKLOADS[name]
+    x = np.ascontiguousarray(latent(name)[w.K])          # the last warm-up snapshot
+    geom = J.Geometry(w.F, w.H, w.W, w.block, w.patch)
+    xd = torch.from_numpy(x).cuda()
+    got = J.fft_scores(xd, geom, cutoff).cpu().numpy()
+    assert J.device_error() == 0
+    ref = oracle.fft_scores(x, w.block, cutoff)
+    err = np.abs(got - ref) - _fft_bound(x, w.block, ref)
+    assert np.all(err <= 0), float(err.max())
+    again = J.fft_scores(xd, geom, cutoff).cpu().numpy()
+    np.testing.assert_array_equal(got.view(np.uint32), again.view(np.uint32))
+
+
+@pytest.mark.parametrize("shape,block", [((2, 3, 9, 12), (1, 4, 4)), ((3, 5, 6, 8), (2, 3, 2)),
+                                         ((1, 1, 16, 16), (1, 2, 2)), ((1, 2, 4, 20), (1, 4, 8)),
+                                         ((4, 3, 19, 21), (1, 8, 8)), ((3, 5, 7, 9), (2, 2, 2)),
+                                         ((2, 5, 10, 13), (2, 4, 4)), ((1, 7, 9, 11), (4, 4, 4)),
+                                         ((2, 3, 7, 11), (1, 4, 4)), ((9, 3, 10, 12), (1, 4, 4)),
+                                         ((6, 2, 9, 10), (2, 4, 4)), ((11, 2, 16, 24), (1, 8, 8))])
+@pytest.mark.parametrize("cutoff", [0, 1, 2, 3])
+def test_fft_scores_edge_geometries(J, shape, block, cutoff):
+    # partial blocks on every axis (FFT lengths below the block's, and edge
+    # lengths 3, 5, 7 that take the direct DFT), each specialised block shape
+    # and the generic one, channel counts below and above the channel groups
+    # (the prefetching walk), unaligned rows (W not a multiple of 4), and
+    # cutoffs from "all bins" (the mean square) to above every folded index
+    # (exactly 0)
+    g = np.random.default_rng(sum(shape) + cutoff)
+    x = (g.standard_normal(shape) * 2.0 + 0.5).astype(np.float32)
+    Cc, F, H, W = shape
+    got = J.fft_scores(torch.from_numpy(x).cuda(), J.Geometry(F, H, W, block, (1, 1, 1)), cutoff)
+    got = got.cpu().numpy()
+    assert J.device_error() == 0
+    ref = oracle.fft_scores(x, block, cutoff)
+    assert np.all(np.abs(got - ref) <= _fft_bound(x, block, ref))
+    assert np.array_equal(got == 0, ref == 0)            # empty bands give exact zeros

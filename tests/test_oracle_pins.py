@@ -585,3 +585,75 @@ def test_literal_and_additive_readings_differ():
     hh = np.arange(8, dtype=np.float32)[None, None, None, :, None] * np.ones((6, 1, 2, 8, 8), np.float32)
     assert np.all(oracle.block_scores_literal(hh, (1, 4, 4)) == 0.0)
     assert np.all(oracle.block_scores(hh, (1, 4, 4))[:2] > 0.0)
+
+
+# ---------------------------------------------------------------- FFT baseline score
+def _blocks(x, block):
+    """Yield (block index, [C][mf][mh][mw] view) in block order."""
+    Cc, F, H, W = x.shape
+    bf, bh, bw = block
+    b = 0
+    for f0 in range(0, F, bf):
+        for h0 in range(0, H, bh):
+            for w0 in range(0, W, bw):
+                yield b, x[:, f0:f0 + bf, h0:h0 + bh, w0:w0 + bw].astype(np.float64)
+                b += 1
+
+
+def _ragged_snapshot(seed):
+    # partial blocks on every axis for the (2, 4, 4) blocks
+    return np.random.default_rng(seed).standard_normal((3, 5, 10, 13)).astype(np.float32) * 1.5 + 0.3
+
+
+@pytest.mark.parametrize("block", [(1, 4, 4), (2, 4, 4), (1, 2, 2), (3, 3, 5)])
+def test_fft_score_cutoff0_is_the_mean_square_by_parseval(block):
+    x = _ragged_snapshot(1)
+    s = oracle.fft_scores(x, block, 0)
+    for b, blk in _blocks(x, block):
+        want = np.mean([np.mean(blk[c] ** 2) for c in range(x.shape[0])])
+        assert s[b] == pytest.approx(want, rel=1e-12)
+
+
+@pytest.mark.parametrize("block", [(1, 4, 4), (2, 4, 4), (1, 2, 2), (3, 3, 5)])
+def test_fft_score_cutoff1_is_the_block_variance_by_parseval(block):
+    # everything but the DC bin: the population variance of each channel's block
+    x = _ragged_snapshot(2)
+    s = oracle.fft_scores(x, block, 1)
+    for b, blk in _blocks(x, block):
+        want = np.mean([np.var(blk[c]) for c in range(x.shape[0])])
+        assert s[b] == pytest.approx(want, rel=1e-10, abs=1e-13)
+
+
+@pytest.mark.parametrize("block,cutoff", [((1, 4, 4), 2), ((2, 4, 4), 1), ((2, 4, 4), 2), ((3, 3, 5), 2),
+                                          ((1, 8, 8), 3)])
+def test_fft_score_matches_library_fft_per_block(block, cutoff):
+    x = np.random.default_rng(3).standard_normal((2, 4, 17, 19)).astype(np.float32)
+    s = oracle.fft_scores(x, block, cutoff)
+    for b, blk in _blocks(x, block):
+        m = blk.shape[1:]
+        fold = [np.abs(np.fft.fftfreq(n) * n).round().astype(int) for n in m]
+        kmax = np.maximum.reduce(np.meshgrid(*fold, indexing="ij"))
+        e = [np.sum(np.abs(np.fft.fftn(blk[c])) ** 2 * (kmax >= cutoff)) for c in range(blk.shape[0])]
+        want = np.mean(e) / np.prod(m) ** 2
+        assert s[b] == pytest.approx(want, rel=1e-10, abs=1e-14)
+
+
+def test_fft_score_planted_frequencies():
+    # a cosine of one cycle per block along h: energy a^2/2, all at folded
+    # index 1; the Nyquist pattern (-1)^h: energy a^2 at folded index 2
+    a = 1.75
+    h = np.arange(8)
+    cos1 = np.broadcast_to((a * np.cos(2 * np.pi * h / 4))[None, None, :, None], (1, 1, 8, 8)).astype(np.float32)
+    nyq = np.broadcast_to((a * (-1.0) ** h)[None, None, :, None], (1, 1, 8, 8)).astype(np.float32)
+    for cutoff, want in ((0, a * a / 2), (1, a * a / 2), (2, 0.0)):
+        np.testing.assert_allclose(oracle.fft_scores(cos1, (1, 4, 4), cutoff), want, atol=1e-12)
+    for cutoff, want in ((1, a * a), (2, a * a), (3, 0.0)):
+        np.testing.assert_allclose(oracle.fft_scores(nyq, (1, 4, 4), cutoff), want, atol=1e-12)
+
+
+def test_fft_score_cutoff_above_every_index_is_zero_and_scores_are_ordered():
+    x = _ragged_snapshot(4)
+    s = [oracle.fft_scores(x, (2, 4, 4), k) for k in range(4)]
+    assert np.all(s[3] == 0.0)
+    for lo, hi in zip(s, s[1:]):
+        assert np.all(hi <= lo + 1e-12)          # a higher cutoff keeps fewer bins
