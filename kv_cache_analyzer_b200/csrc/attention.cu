@@ -10,7 +10,9 @@
 // (pair of 128-query tiles, head); 12 warps:
 //   warps 0-3, 4-7  softmax warpgroups WG0 / WG1, one per query tile:
 //              thread = one query row = one TMEM lane.  Per key tile the row's
-//              S (128 fp32) is read from TMEM in two halves, the running max
+//              S (128 fp32) is read from TMEM in one round trip (setmaxnreg
+//              moves registers from warps 8-11 to these two warpgroups so
+//              the whole row fits), the running max
 //              is kept in the log2 domain and O is rescaled in TMEM only when
 //              the max grows by more than 2^8 (lazy rescale), P is written as
 //              packed BF16 into the upper half of the row's S columns (keys
@@ -29,7 +31,7 @@
 //              from smem.  tcgen05.commit hands S to the softmax warps and
 //              frees ring slots.  Because S_i_j is issued after PV_i_{j-1},
 //              the softmax that sees S_i_j may rescale O_i safely.
-//   warps 10-11 idle.
+//   warps 10-11 idle (with 8-9 they form the warpgroup that gives up registers).
 // TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [384,384+d);
 // P_i occupies columns [64,128) of S_i.
 // Every wait is bounded; on timeout the CTA records JANO_ETIMEOUT, drains its
@@ -49,6 +51,17 @@ constexpr int BM = 128;            // queries per tile (two tiles per CTA)
 constexpr int BN = 128;            // keys per tile
 constexpr int kSlots = 4;          // K/V ring slots
 constexpr int kThreads = 384;
+// Registers per thread: at launch (384 x 168 = 64,512), then rebalanced:
+// the producer / MMA warpgroup (warps 8-11) drops to kRegsIssue and the two
+// softmax warpgroups rise to kRegsSoftmax, so that a softmax thread holds
+// its whole 128-column S row.  2 x 128 x 208 + 128 x 80 = 63,488 of the
+// 64,512, and per SM sub-partition (one warp of each warpgroup)
+// 208 + 208 + 80 = 496 of 512.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsIssue = 80;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIssue <= kThreads * kRegsLaunch, "register split");
+static_assert(2 * kRegsSoftmax + kRegsIssue <= 512, "sub-partition register file");
 constexpr uint32_t kPanel = 128 * 128;   // bytes of one 128-row x 64-col BF16 panel
 constexpr long long kWaitLimit = 1ll << 31;  // cycles (~1 s)
 
@@ -108,12 +121,6 @@ struct Ctl {
     }
 };
 
-// 64 consecutive TMEM columns of this warp's 32 lanes into registers.
-__device__ __forceinline__ void ld64(uint32_t taddr, uint32_t (&r)[64]) {
-    ptx::tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-    ptx::tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-}
-
 // Row max of 64 values (8 independent chains of 3-input max); with kMask,
 // keys >= valid (the ragged last key tile) are left out.
 template <bool kMask>
@@ -163,9 +170,9 @@ __device__ __forceinline__ void exp2_poly2(uint64_t x2, float& ya, float& yb) {
 }
 
 // Share of the exponentials computed by exp2_poly2, in eighths: pairs whose
-// index modulo 8 is below this count (0 = all on MUFU, 2 = a quarter).
+// index modulo 8 is below this count (0 = all on MUFU, 1 = an eighth).
 #ifndef JANO_EXP2_POLY_EIGHTHS
-#define JANO_EXP2_POLY_EIGHTHS 2
+#define JANO_EXP2_POLY_EIGHTHS 1
 #endif
 
 // p = 2^(s*c - m) for 64 values, packed to 32 BF16x2 words; returns sum(p).
@@ -197,19 +204,21 @@ __device__ __forceinline__ float exp64(const uint32_t (&s)[64], int valid, float
     return lo + hi;
 }
 
-// One key tile of one query row: row max over S (TMEM, two 64-column
-// halves), lazy O rescale, P = 2^(S*c - m) as BF16 into the upper half of
-// the row's S columns.  Warp-uniform control flow throughout.
+// One key tile of one query row: the row's 128 S values from TMEM in one
+// round trip, row max, lazy O rescale, P = 2^(S*c - m) as BF16 into the upper
+// half of the row's S columns.  Warp-uniform control flow throughout.
 template <int HD, bool kMask>
 __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, uint32_t tP, int j, int valid,
                                              float c, float& m, float& l, uint32_t bar_half) {
-    uint32_t s[64];
-    ld64(tS, s);
+    uint32_t s[128];
+    ptx::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+    ptx::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+    ptx::tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+    ptx::tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
     ptx::tmem_wait_ld();
-    float mx = max64<kMask>(s, valid);
-    ld64(tS + 64, s);
-    ptx::tmem_wait_ld();
-    mx = fmaxf(mx, max64<kMask>(s, valid - 64));
+    const uint32_t(&lo)[64] = *reinterpret_cast<const uint32_t(*)[64]>(&s[0]);
+    const uint32_t(&hi)[64] = *reinterpret_cast<const uint32_t(*)[64]>(&s[64]);
+    const float mx = fmaxf(max64<kMask>(lo, valid), max64<kMask>(hi, valid - 64));
     const float mxs = mx * c;
     // lazy rescale, decided per warp so the TMEM accesses stay warp-wide:
     // lanes whose max did not grow past 2^8 keep their max (alpha = 1).
@@ -227,10 +236,10 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, uint32_t 
                 const uint64_t a2 = ptx::f2(alpha, alpha);
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    float lo, hi;
-                    ptx::f2split(ptx::fmul2(ptx::f2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), lo, hi);
-                    o[e] = __float_as_uint(lo);
-                    o[e + 1] = __float_as_uint(hi);
+                    float lo2, hi2;
+                    ptx::f2split(ptx::fmul2(ptx::f2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), lo2, hi2);
+                    o[e] = __float_as_uint(lo2);
+                    o[e + 1] = __float_as_uint(hi2);
                 }
                 ptx::tmem_st32(tO + 32 * q, o);
             }
@@ -238,19 +247,16 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, uint32_t 
         }
         m = m_new;
     }
-    // the upper half is still in registers: its P goes to P columns [32,64)
+    // upper key half first: its P goes to P columns [32,64) and is handed to
+    // the MMA thread, whose P.V runs while the lower half is exponentiated
     uint32_t pk[32];
-    l += exp64<kMask>(s, valid - 64, c, m, pk);
+    l += exp64<kMask>(hi, valid - 64, c, m, pk);
     ptx::tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(pk));
-    // hand the upper key half to the MMA thread now: its P.V runs while the
-    // lower half's exponentials are computed
     ptx::tmem_wait_st();
     ptx::tc_fence_before();
     __syncwarp();
     if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(bar_half);
-    ld64(tS, s);
-    ptx::tmem_wait_ld();
-    l += exp64<kMask>(s, valid, c, m, pk);
+    l += exp64<kMask>(lo, valid, c, m, pk);
     ptx::tmem_st32(tP, *reinterpret_cast<uint32_t(*)[32]>(pk));
     ptx::tmem_wait_st();
 }
@@ -307,7 +313,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 8) {
+    if (warp >= 8) {
+      ptx::setmaxnreg_dec<kRegsIssue>();
+      if (warp == 8) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             int last[kSlots];
@@ -411,7 +419,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
             ptx::mma_commit(ctl.bar(L::bFinal));
             ptx::mbar_wait(ctl.bar(L::bFinal), 0, kWaitLimit);
         }
-    } else if (warp < 8) {
+      }
+    } else {
+        ptx::setmaxnreg_inc<kRegsSoftmax>();
         // ------------------------------------------------------------ softmax WG i
         const int i = warp >> 2;                      // query tile of this warpgroup
         const int q = warp & 3;                       // TMEM lane quarter of this warp
@@ -508,8 +518,14 @@ cudaError_t launch_hd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !(done_mask & (1ull << dev))) {
-        cudaError_t e = cudaFuncSetAttribute(attention_kernel<HD>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc);
+        // the register split assumes exactly kRegsLaunch registers per thread
+        // at launch; anything else could leave an increase waiting for good
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, attention_kernel<HD>);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
+        e = cudaFuncSetAttribute(attention_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)L::kAlloc);
         if (e != cudaSuccess) return e;
         if (dev < 64) done_mask |= 1ull << dev;
     }

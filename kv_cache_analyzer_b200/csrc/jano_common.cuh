@@ -241,6 +241,19 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
 }
 
 // Hardware square root approximation (relative error about 2^-22).
+// Register rebalancing between warpgroups (all four warps of a warpgroup
+// execute it).  The counts must add up, over the CTA's warpgroups, to at
+// most the registers the CTA was launched with, or an increase waits for
+// good; the launchers check the launch register count before using it.
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ float sqrt_approx(float x) {
     float y;
     asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
