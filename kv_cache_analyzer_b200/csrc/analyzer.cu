@@ -393,15 +393,15 @@ cudaError_t launch_block_scores(const float* lat, int K, int C, const jano_geom&
         return cudaErrorInvalidValue;
 
     const size_t smem = (size_t)a.smem;
-    static unsigned long long done_mask[2] = {0, 0};   // per-device shared-memory opt-in
+    static DeviceOnce opted_in[2];   // per-device shared-memory opt-in, per instantiation
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (dev >= 64 || !(done_mask[literal] & (1ull << dev))) {
+    if (!opted_in[literal].done(dev)) {
         cudaError_t e = cudaFuncSetAttribute(literal ? analyzer_kernel<true> : analyzer_kernel<false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, 224 * 1024);
         if (e != cudaSuccess) return e;
-        if (dev < 64) done_mask[literal] |= 1ull << dev;
+        opted_in[literal].mark(dev);
     }
     const int threads = a.NC + 32;
     // resident CTAs per SM: shared memory (228 KB, 1 KB reserved per CTA) and threads

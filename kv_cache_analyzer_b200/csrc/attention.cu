@@ -514,10 +514,10 @@ cudaError_t launch_hd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
                       void* out, int* err, cudaStream_t st) {
     using L = Layout<HD>;
     // the shared-memory opt-in is per device: remember which devices have it
-    static unsigned long long done_mask = 0;
+    static DeviceOnce ready;
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 64 || !(done_mask & (1ull << dev))) {
+    if (!ready.done(dev)) {
         // the register split assumes exactly kRegsLaunch registers per thread
         // at launch; anything else could leave an increase waiting for good
         cudaFuncAttributes fa;
@@ -527,7 +527,7 @@ cudaError_t launch_hd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
         e = cudaFuncSetAttribute(attention_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)L::kAlloc);
         if (e != cudaSuccess) return e;
-        if (dev < 64) done_mask |= 1ull << dev;
+        ready.mark(dev);
     }
     const int q_tiles = (n_act + BM - 1) / BM;
     const dim3 grid((q_tiles + 1) / 2, heads);

@@ -213,14 +213,14 @@ cudaError_t launch_classify(const float* scores, int n, long long k_static,
                             cudaStream_t st) {
     const int per_cta = (n + kCluster - 1) / kCluster;
     const size_t smem = per_cta <= kMaxCachedKeys ? (size_t)per_cta * 4 : 0;
-    static unsigned long long done_mask = 0;   // per-device shared-memory opt-in
+    static DeviceOnce opted_in;   // per-device shared-memory opt-in
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 64 || !(done_mask & (1ull << dev))) {
+    if (!opted_in.done(dev)) {
         cudaError_t e = cudaFuncSetAttribute(classify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kMaxCachedKeys * 4);
         if (e != cudaSuccess) return e;
-        if (dev < 64) done_mask |= 1ull << dev;
+        opted_in.mark(dev);
     }
     classify_kernel<<<kCluster, kThreads, smem, st>>>(reinterpret_cast<const uint32_t*>(scores), n,
                                                       k_static, k_active, levels, err);

@@ -12,15 +12,19 @@ namespace jano {
 __device__ int g_device_error = JANO_OK;
 
 int* device_error_word() {
-    static int* addr[64] = {nullptr};
+    // cached per device; several host threads may fill a slot, all with the
+    // same address
+    static std::atomic<int*> addr[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!addr[dev]) {
+    int* a = addr[dev].load(std::memory_order_acquire);
+    if (!a) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-        addr[dev] = static_cast<int*>(p);
+        a = static_cast<int*>(p);
+        addr[dev].store(a, std::memory_order_release);
     }
-    return addr[dev];
+    return a;
 }
 
 namespace {

@@ -6,6 +6,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 #include "../../include/jano.h"
@@ -22,6 +23,23 @@ __device__ __forceinline__ void raise_error(int* err, int code) {
 }
 
 int* device_error_word();   // address of this device's error word (host)
+
+// Per-device "set up once" flags for host-side launch preparation (the
+// shared-memory opt-in of a kernel, a launch-attribute check), safe to use
+// from several host threads.  Devices 64 and up are never marked done, so
+// their set-up simply runs on every launch.
+class DeviceOnce {
+  public:
+    bool done(int dev) const {
+        return dev >= 0 && dev < 64 && ((mask_.load(std::memory_order_acquire) >> dev) & 1ull);
+    }
+    void mark(int dev) {
+        if (dev >= 0 && dev < 64) mask_.fetch_or(1ull << dev, std::memory_order_release);
+    }
+
+  private:
+    std::atomic<unsigned long long> mask_{0};
+};
 
 // Launchers implemented by the kernel translation units.  They assume the
 // arguments were validated by the exported entry points.

@@ -372,14 +372,14 @@ cudaError_t launch_bn(const void* w, const GemmArgs& a, cudaStream_t st) {
     using L = PLayout<BN>;
     CUtensorMap mB;
     if (!make_map2d(&mB, w, a.n, a.k, BN)) return cudaErrorInvalidValue;
-    static unsigned long long done_mask = 0;   // per-device shared-memory opt-in
+    static DeviceOnce opted_in;   // per-device shared-memory opt-in
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 64 || !(done_mask & (1ull << dev))) {
+    if (!opted_in.done(dev)) {
         cudaError_t e = cudaFuncSetAttribute(projection_kernel<BN>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc);
         if (e != cudaSuccess) return e;
-        if (dev < 64) done_mask |= 1ull << dev;
+        opted_in.mark(dev);
     }
     const int tiles = ((a.m + PM - 1) / PM) * ((a.n + BN - 1) / BN);
     int sms = 148;
