@@ -39,10 +39,13 @@ def frame_block_range(rank: int, world: int, n_fb: int) -> tuple[int, int]:
 
 
 def slab_frames(rank: int, world: int, F: int, bf: int) -> tuple[int, int, int]:
-    """(first frame, frames owned, frames in the slab incl. the halo frame)."""
+    """(first frame, frames owned, frames in the slab incl. the halo frame);
+    a rank that owns no frame-block gets an empty slab."""
     n_fb = -(-F // bf)
     lo, hi = frame_block_range(rank, world, n_fb)
     f0, f1 = lo * bf, min(hi * bf, F)
+    if f1 == f0:
+        return f0, 0, 0
     halo = 1 if f1 < F else 0
     return f0, f1 - f0, f1 - f0 + halo
 
@@ -137,9 +140,11 @@ class ShardedHotPath:
 
     # ------------------------------------------------------------------ step
     def run_local_scores(self):
-        """a1 on this rank's slab (its own blocks first, the halo frame's last)."""
-        jano_block_scores(self.lat, self.K, self.C, self._sgc, self.w_t, self.w_s,
-                          self.slab_scores, self.stream)
+        """a1 on this rank's slab (its own blocks first, the halo frame's last);
+        nothing when the rank owns no frame-block (more ranks than blocks)."""
+        if self.n_local:
+            jano_block_scores(self.lat, self.K, self.C, self._sgc, self.w_t, self.w_s,
+                              self.slab_scores, self.stream)
 
     def local_scores(self) -> torch.Tensor:
         return self.slab_scores[:self.n_local]
@@ -168,9 +173,12 @@ class ShardedHotPath:
         return o[step], o[step + 1] - o[step]
 
     def run_head_kernels(self, step: int):
-        """a4, a5 of sampling step `step` on this rank's heads."""
+        """a4, a5 of sampling step `step` on this rank's heads (none when the
+        rank owns no head: more ranks than heads)."""
         s = self.stream
         start, n_act = self.due(step)
+        if self.heads == 0:
+            return n_act
         idx = self.idx[start:start + n_act]
         jano_kv_scatter(self.k_act, self.v_act, idx, n_act, self.heads, self.d,
                         self.k_cache, self.v_cache, self.N, s)

@@ -25,8 +25,12 @@ def _bits(t):
     return t.contiguous().view(torch.int16 if t.dtype == torch.bfloat16 else torch.int32).cpu()
 
 
-@pytest.mark.parametrize("name,world", [("tiny", 2), ("small", 2), ("small", 3), ("large", 8)])
+@pytest.mark.parametrize("name,world", [("tiny", 2), ("small", 2), ("small", 3), ("large", 8),
+                                        ("small", 5), ("image", 3), ("tiny", 8)])
 def test_sharded_step_equals_unsharded(name, world):
+    # uneven shares (12 heads and 21 frames over 5 ranks), ranks without a
+    # frame-block (one frame over 3 ranks) and ranks without a head or a
+    # frame-block (4 heads and 4 frames over 8 ranks) included
     import bench
     import synth
     import kv_cache_analyzer_b200 as J

@@ -68,7 +68,7 @@ def test_partitions_cover_everything_once():
             for r in range(world):
                 f0, own, slab = slab_frames(r, world, F, bf)
                 frames += list(range(f0, f0 + own))
-                assert slab == own + (1 if f0 + own < F else 0)
+                assert slab == (own + (1 if f0 + own < F else 0) if own else 0)
             assert frames == list(range(F))
 
 
@@ -90,7 +90,10 @@ def _shard_worker(rank, world, port, out):
                   for r in range(world)]
         # this rank's blocks, scored on its slab with the halo frame (the oracle
         # stands in for the kernel on the CPU ranks)
-        local = torch.from_numpy(oracle.block_scores(np.ascontiguousarray(lat[:, :, f0:f0 + slab]), block))
+        if slab:
+            local = torch.from_numpy(oracle.block_scores(np.ascontiguousarray(lat[:, :, f0:f0 + slab]), block))
+        else:
+            local = torch.zeros(0, dtype=torch.float64)         # a rank without frame-blocks
         full = torch.empty(sum(counts), dtype=torch.float64)
         torch_all_gather(local[:counts[rank]].contiguous(), full, counts)
         out[rank] = full.numpy().tobytes()
@@ -99,7 +102,7 @@ def _shard_worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 7])
 def test_sharded_scores_gather_to_the_whole_latent(world):
     # frame slabs with one halo frame, scored per rank and all-gathered, give
     # the scores of the whole latent exactly (uneven slabs with 3 ranks)
