@@ -258,7 +258,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
          | ((uint32_t)(M >> 4) << 24);
 }
 
-// Hardware square root approximation (relative error about 2^-22).
 // Register rebalancing between warpgroups (all four warps of a warpgroup
 // execute it).  The counts must add up, over the CTA's warpgroups, to at
 // most the registers the CTA was launched with, or an increase waits for
@@ -272,6 +271,7 @@ __device__ __forceinline__ void setmaxnreg_dec() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// Hardware square root approximation (relative error about 2^-22).
 __device__ __forceinline__ float sqrt_approx(float x) {
     float y;
     asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
