@@ -153,9 +153,9 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ traffic record
-def traffic_for(kernel_src_rel):
+def traffic_for(kernel_src_rel, workload):
     """DRAM bytes per launch from the committed ncu record, if it was taken on
-    the current source of that kernel; else None."""
+    the current source of that kernel and on this workload; else None."""
     rec = os.path.join(ROOT, "profiles", "traffic.json")
     src = os.path.join(ROOT, kernel_src_rel)
     if not (os.path.exists(rec) and os.path.exists(src)):
@@ -166,7 +166,9 @@ def traffic_for(kernel_src_rel):
     if not ent:
         return None
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return ent.get("bytes_per_launch") if ent.get("source_sha") == sha else None
+    if ent.get("source_sha") != sha or ent.get("workload_key") != workload:
+        return None
+    return ent.get("bytes_per_launch")
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -463,7 +465,7 @@ def run_gpu(args, w, rank, world, local_rank, dist):
     kernels["active_attention"]["frac_of_burst_peak"] = att_tflops / pk["bf16_tflops"]
     roofline = {"bound": "tensor", "achieved": att_tflops, "peak": bf16_sus, "unit": "TFLOP/s",
                 "frac": att_tflops / bf16_sus,
-                "traffic": traffic_for("kv_cache_analyzer_b200/csrc/attention.cu"),
+                "traffic": traffic_for("kv_cache_analyzer_b200/csrc/attention.cu", w.name),
                 "peak_kind": f"{pk_src} sustained cuBLAS bf16 (kernel timed inside a long step)",
                 "kernel": "active_attention"}
 
@@ -482,9 +484,11 @@ def run_gpu(args, w, rank, world, local_rank, dist):
         next_rows.update(measure_fft_score(J, hp, stream, pk))
 
     cfg = workload_config(w)
+    cache_gb = 2.0 * w.n_tokens * w.heads * w.d * 2 / 1e9
+    act_gb = 3.0 * n_cap * w.heads * w.d * 2 / 1e9
     cfg.update({"n_active": n_act, "global_batch": world, "parallelism": f"replicas x{world}",
-                "l2": "no flush: the per-step working set (K/V cache 1.5 GB, Q/K/V act 0.6 GB) "
-                      "is far larger than the 126 MB L2"})
+                "l2": f"no flush: the per-step working set (K/V cache {cache_gb:.2f} GB, Q/K/V act "
+                      f"{act_gb:.2f} GB) is larger than the 126 MB L2"})
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
