@@ -1,10 +1,12 @@
 """Per-rank work of the head-sharded step, measured one rank at a time.
 
     python -m kv_cache_analyzer_b200.sharding_run [--ranks 1 2 4 8] [--reps R]
+        [--frames F] [--height H] [--width W] [--heads N]
 
-Builds the step of the large video workload (latent [6][16][21][90][160]
-fp32 with 1x4x4 blocks, 75,600 tokens x 40 heads x d=128 BF16, 25/30/45
-level split, first interleaved step = the 18,900 Active tokens) from random
+Builds the step of the large video workload by default (latent
+[6][16][21][90][160] fp32 with 1x4x4 blocks, 75,600 tokens x 40 heads x
+d=128 BF16, 25/30/45 level split, first interleaved step = the 18,900
+Active tokens; the size flags shrink it) from random
 device inputs, cuts it into W ranks with ``ShardedHotPath`` (frame slabs for
 the analyzer, head ranges for scatter and attention) and times each rank's
 kernels alone on this GPU with CUDA events: its block scores, then (after the
@@ -43,9 +45,13 @@ def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--ranks", type=int, nargs="+", default=[1, 2, 4, 8])
     ap.add_argument("--reps", type=int, default=5)
+    ap.add_argument("--frames", type=int, default=21)
+    ap.add_argument("--height", type=int, default=90)
+    ap.add_argument("--width", type=int, default=160)
+    ap.add_argument("--heads", type=int, default=40)
     args = ap.parse_args(argv)
-    K, C, F, H, W = 5, 16, 21, 90, 160
-    heads, d = 40, 128
+    K, C, F, H, W = 5, 16, args.frames, args.height, args.width
+    heads, d = args.heads, 128
     frac_active, frac_static = 0.25, 0.45
     lg = Geometry(F, H, W, (1, 4, 4), (1, 2, 2))
     tg = Geometry(F, H, W, (1, 2, 2), (1, 2, 2))
