@@ -98,11 +98,14 @@ struct Ctl {
     volatile int* abort;
     int* err;
     __device__ uint32_t bar(int i) const { return bar0 + 8u * (uint32_t)i; }
+    // Waiting threads are suspended (not spinning) until the phase completes,
+    // leaving the issue slots to the softmax warps that share their
+    // sub-partition.
     __device__ bool wait(int i, uint32_t parity) const {
-        if (ptx::mbar_try_wait(bar(i), parity)) return true;
+        if (ptx::mbar_try_wait_sleep(bar(i), parity)) return true;
         const long long t0 = clock64();
         for (;;) {
-            if (ptx::mbar_try_wait(bar(i), parity)) return true;
+            if (ptx::mbar_try_wait_sleep(bar(i), parity)) return true;
             if (*abort) return false;
             if (clock64() - t0 > kWaitLimit) {
                 *abort = 1;
