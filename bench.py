@@ -283,34 +283,38 @@ def measure_projections(J, hp, step, stream, pk, reps=10, cpu_rows=0):
 
 def measure_fft_score(J, hp, stream, pk, reps=10, cutoff=1):
     """The FFT baseline score (outside the step, reported beside it) against
-    the analyzer under the same conditions: each launch alone, L2 flushed
-    before it (a 256 MB write), on the last warm-up snapshot x_K.  The FFT
-    score reads one snapshot; the analyzer reads all K+1."""
+    the analyzer under the same conditions: each launch alone, L2 cleaned
+    before it (a 256 MB read, which leaves no dirty lines to write back), on
+    the last warm-up snapshot x_K.  The FFT score reads one snapshot; the
+    analyzer reads all K+1.  A plain torch.sum over the analyzer's bytes,
+    timed the same way, gives the rate a single pass of that size reaches."""
     import torch
     K, C = hp.K, hp.C
     x = hp.lat[K]
     out = torch.empty_like(hp.scores)
     geom = hp.lg.c()
-    flush = torch.empty(64 << 20, dtype=torch.float32, device=hp.dev)
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=hp.dev)
     snap_bytes = float(x.numel()) * 4 + out.numel() * 4
     lat_bytes = float(hp.lat.numel()) * 4 + out.numel() * 4
     ops = {
         "fft_score": (lambda: J.jano_fft_scores(x, C, geom, cutoff, out, stream), snap_bytes),
         "block_scores_same_conditions": (lambda: J.jano_block_scores(hp.lat, K, C, geom, hp.w_t, hp.w_s,
                                                                      out, stream), lat_bytes),
+        "plain_read_same_bytes": (lambda: torch.sum(hp.lat), float(hp.lat.numel()) * 4),
     }
     res = {}
     for name, (fn, nbytes) in ops.items():
-        for _ in range(3):
-            fn()
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
         ms = []
         for _ in range(reps):
             with torch.cuda.stream(stream):
-                flush.fill_(1.0)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            fn()
-            b.record(stream)
+                flush.sum()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
             stream.synchronize()
             ms.append(a.elapsed_time(b))
         m = sorted(ms)[reps // 2]

@@ -5,10 +5,11 @@
 
 A random fp32 latent history [K+1][C][F][H][W] (N(0, 1)) on the device.
 Times, with CUDA events on the current stream after three warm-up calls and
-with the L2 flushed (a 256 MB write) before every launch, the FFT score of
-the last snapshot (jano_fft_scores: one snapshot read) and the analyzer's
-block scores (jano_block_scores: all K+1 snapshots read), and prints one JSON
-line with each launch's time and HBM GB/s over its algorithmic bytes.
+with the L2 cleaned (a 256 MB read) before every launch, the FFT score of
+the last snapshot (jano_fft_scores: one snapshot read), the analyzer's block
+scores (jano_block_scores: all K+1 snapshots read) and, for scale, a plain
+torch.sum over the analyzer's bytes, and prints one JSON line with each
+launch's time and HBM GB/s over its algorithmic bytes.
 Defaults: the large video latent (C=16, 21 x 90 x 160, 1x4x4 blocks, K=5).
 """
 from __future__ import annotations
@@ -38,14 +39,15 @@ def main(argv=None):
     lat = torch.randn((K + 1, C, F, H, W), generator=g, device=dev)
     geom = Geometry(F, H, W, tuple(args.block), (1, 1, 1))
     out = torch.empty(geom.n_blocks, device=dev)
-    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
     st = torch.cuda.current_stream()
     gc = geom.c()
     snap = lat[K]
     ops = {"fft_score": (lambda: jano_fft_scores(snap, C, gc, args.cutoff, out, st),
                          4.0 * (snap.numel() + out.numel())),
            "block_scores": (lambda: jano_block_scores(lat, K, C, gc, 0.5, 0.5, out, st),
-                            4.0 * (lat.numel() + out.numel()))}
+                            4.0 * (lat.numel() + out.numel())),
+           "plain_read": (lambda: torch.sum(lat), 4.0 * lat.numel())}
     res = {"shape": {"channels": C, "frames": F, "height": H, "width": W, "block": list(args.block),
                      "steps": K, "cutoff": args.cutoff, "n_blocks": geom.n_blocks}}
     for name, (fn, nbytes) in ops.items():
@@ -53,7 +55,7 @@ def main(argv=None):
             fn()
         ms = []
         for _ in range(args.reps):
-            flush.fill_(1.0)
+            flush.sum()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(st)
             fn()

@@ -25,7 +25,7 @@ def test_spectral_run(capsys):
     spectral_run.main(["--channels", "4", "--frames", "3", "--height", "18", "--width", "40", "--reps", "2"])
     (d,) = _lines(capsys)
     assert d["shape"]["n_blocks"] == 3 * 5 * 10
-    assert d["fft_score"]["GB/s"] > 0 and d["block_scores"]["GB/s"] > 0
+    assert d["fft_score"]["GB/s"] > 0 and d["block_scores"]["GB/s"] > 0 and d["plain_read"]["GB/s"] > 0
 
 
 def test_sharding_run(capsys):
