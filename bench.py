@@ -17,8 +17,9 @@ has no data-path exchange, so N GPUs process N problems ("weak" scaling).
 Beside the step (not in its value) the line reports ``next_rows``: the
 block's projections on the step's active tokens -- the fused Q/K/V projection
 writing K/V straight into the cache and the output projection scattered back
-to the token rows -- with their TFLOP/s, and the FFT baseline score with
-the analyzer timed under the same conditions (HBM GB/s).
+to the token rows -- with their TFLOP/s, the FFT baseline score with the
+analyzer timed under the same conditions (HBM GB/s), and the attention at
+the schedule's larger due sets (Active + Moderate, and every token).
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead, on
 a bounded sample of the same workload, extrapolated stage by stage to the
@@ -281,6 +282,45 @@ def measure_projections(J, hp, step, stream, pk, reps=10, cpu_rows=0):
     return res
 
 
+def measure_attention_sizes(J, hp, stream, pk, reps=3):
+    """Attention over the same cache at the step's larger due sets (outside
+    the step, reported beside it): an interleaved step where Active and
+    Moderate tokens are due, and a full step (every token due, e.g. warm-up),
+    with random BF16 queries.  TFLOP/s as for the headline."""
+    import torch
+    N, H, d = hp.N, hp.heads, hp.d
+    o = hp.host_offsets
+    step_am = next((t for t in range(hp.sched.warmup, hp.sched.T - hp.sched.cooldown)
+                    if o[t + 1] - o[t] > o[hp.sched.warmup + 1] - o[hp.sched.warmup]), None)
+    cases = {"full": (0, o[1] - o[0])}
+    if step_am is not None:
+        cases["active_moderate"] = (o[step_am], o[step_am + 1] - o[step_am])
+    g = torch.Generator(device=hp.dev).manual_seed(4321)
+    q = torch.randn((N, H, d), generator=g, device=hp.dev).to(torch.bfloat16)
+    out = torch.empty((N, H, d), dtype=torch.bfloat16, device=hp.dev)
+    res = {}
+    for name, (start, n) in cases.items():
+        idx = hp.idx[start:start + n]
+        qn = q[:n]
+        fn = lambda: J.jano_active_attention(qn, hp.k_cache, hp.v_cache, idx, n, N, H, d, d ** -0.5, out, stream)
+        fn()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        evs[0].record(stream)
+        for i in range(reps):
+            fn()
+            evs[i + 1].record(stream)
+        stream.synchronize()
+        ms = sorted(evs[i].elapsed_time(evs[i + 1]) for i in range(reps))[reps // 2]
+        flops = 4.0 * n * N * d * H
+        tf = flops / (ms * 1e-3) / 1e12
+        res[f"attention_{name}"] = {"ms": ms, "TFLOP/s": tf, "n_active": n, "flops": flops,
+                                    "frac_of_sustained_peak": tf / pk.get("bf16_tflops_sustained", pk["bf16_tflops"])}
+    code = J.device_error(stream)
+    if code:
+        raise RuntimeError(f"device error in the attention sizes: {J.jano_status_str(code)}")
+    return res
+
+
 def measure_fft_score(J, hp, stream, pk, reps=10, cutoff=1):
     """The FFT baseline score (outside the step, reported beside it) against
     the analyzer under the same conditions: each launch alone, L2 cleaned
@@ -486,6 +526,7 @@ def run_gpu(args, w, rank, world, local_rank, dist):
         next_rows = measure_projections(J, hp, step, stream, pk,
                                         cpu_rows=0 if args.no_cpu_baseline or world > 1 else 2)
         next_rows.update(measure_fft_score(J, hp, stream, pk))
+        next_rows.update(measure_attention_sizes(J, hp, stream, pk))
 
     cfg = workload_config(w)
     cache_gb = 2.0 * w.n_tokens * w.heads * w.d * 2 / 1e9
