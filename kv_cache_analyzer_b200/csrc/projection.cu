@@ -7,27 +7,31 @@
 //
 //   out_seg(r)[dst_seg(r)][j] = sum_c x[src(r)][c] * w[j][c]
 //
-// A persistent grid, one CTA per SM, walks the 128-row x BN-column output
-// tiles; 9 warps:
-//   warps 0-3  producers.  The tile's 128 source rows (src(r) = gather[r],
+// A persistent grid, one CTA per SM, walks the 256-row x BN-column output
+// tiles (two 128-row MMA halves that share every weight stage, which cuts
+// the shared-memory traffic per FLOP: an SS MMA reads both operands from
+// shared memory at 128 B/clk); 9 warps:
+//   warps 0-3  producers.  The tile's 256 source rows (src(r) = gather[r],
 //            or r) are read once into shared memory.  Per 64-column K block
 //            the A rows are gathered with 16-byte cp.async copies (eight
 //            lanes per 128-byte row, zero-filled for rows past m), written
 //            straight into the 128-byte-swizzled K-major layout the tensor
 //            core reads (chunk c of row i at i*128 + ((c ^ (i % 8)) * 16));
-//            the weight rows come by one tiled TMA box.  A 4-slot ring; each
+//            the weight rows come by one tiled TMA box.  A 3-slot ring; each
 //            producer thread hands a stage over with cp.async.mbarrier.arrive
 //            (the barrier cannot complete before that thread's copies have
 //            landed) plus an ordinary arrive, so it never waits for its own
 //            copies and runs as far ahead as the ring allows.
-//   warp 4   allocates 2 x BN TMEM columns (two accumulators); one lane
-//            issues tcgen05.mma (kind::f16, M=128, N=BN, K=16, both operands
-//            K-major from shared memory, fp32 accumulator in TMEM) into the
-//            accumulators in turn and frees ring slots with tcgen05.commit.
-//   warps 5-8  epilogue: thread = one output row = one TMEM lane; a tile's
-//            accumulator (ready while the next tile's MMAs fill the other
-//            one) is read 32 columns at a time, rounded to BF16 and
-//            stored to the row's destination.  The N range may be cut into
+//   warp 4   allocates the 512 TMEM columns; one lane issues tcgen05.mma
+//            (kind::f16, M=128, N=BN, K=16, both operands K-major from
+//            shared memory, fp32 accumulators in TMEM), two per K slice (one
+//            per half of the tile), and frees ring slots with
+//            tcgen05.commit.  For BN = 256 one accumulator set (2 x 256
+//            columns) fills TMEM; for BN = 128 two sets alternate, so the
+//            epilogue overlaps the next tile.
+//   warps 5-8  epilogue: thread = one TMEM lane = one row of each half; a
+//            tile's accumulators are read 32 columns at a time, rounded to
+//            BF16 and stored to the rows' destinations.  The N range may be cut into
 //            segments with their own destination and row map, which is how
 //            the fused Q/K/V projection writes Q to the active rows and K, V
 //            straight into the token-ordered KV cache.
@@ -46,9 +50,9 @@
 namespace jano {
 namespace {
 
-constexpr int PM = 128;                 // output rows per CTA
+constexpr int PM = 256;                 // output rows per tile (two 128-row MMA halves)
 constexpr int PK = 64;                  // K columns per stage (128 bytes of BF16)
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kProducers = 128;         // warps 0-3
 constexpr int kMmaWarp = 4;
 constexpr int kThreads = 288;
@@ -73,7 +77,10 @@ struct GemmArgs {
 
 template <int BN>
 struct PLayout {
-    static constexpr uint32_t kA = PM * PK * 2;                  // 16 KB
+    // accumulator sets in TMEM (each: two halves of BN columns): two when
+    // they fit in the 512 columns, so the epilogue overlaps the next tile
+    static constexpr int kAccBuf = 4 * BN <= 512 ? 2 : 1;
+    static constexpr uint32_t kA = PM * PK * 2;                  // 32 KB
     static constexpr uint32_t kB = BN * PK * 2;                  // 32 KB for BN = 256
     static constexpr uint32_t kStage = kA + kB;
     static constexpr uint32_t kBar = kStages * kStage;
@@ -181,7 +188,7 @@ projection_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
         ptx::fence_mbar_init();
     }
     if (warp == kMmaWarp) {
-        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), 2 * BN);
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), 512);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
@@ -255,26 +262,30 @@ projection_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = ptx::idesc_bf16(PM, BN, false, false);
+            constexpr uint32_t idesc = ptx::idesc_bf16(128, BN, false, false);
             int q = 0, lt = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x, ++lt) {
-                const int b = lt & 1;
-                // the epilogue has read this accumulator's previous tile
-                if (!ctl.wait(L::bAccEmpty + b, ((lt >> 1) & 1) ^ 1)) { ok = false; break; }
+                const int b = lt % L::kAccBuf;
+                // the epilogue has read this accumulator set's previous tile
+                if (!ctl.wait(L::bAccEmpty + b, ((lt / L::kAccBuf) & 1) ^ 1)) { ok = false; break; }
                 ptx::tc_fence_after();
-                const uint32_t acc = tmem + b * BN;
+                const uint32_t acc = tmem + b * 2 * BN;       // rows 0-127; rows 128-255 at + BN
                 for (int kb = 0; kb < nkb; ++kb, ++q) {
                     const int s = q % kStages;
                     if (!ctl.wait(L::bFull + s, (q / kStages) & 1)) { ok = false; break; }
                     fence_proxy_async();
                     ptx::tc_fence_after();
                     const uint32_t sa = base + s * L::kStage;
+                    // both 128-row halves of A against the same B stage
 #pragma unroll
-                    for (int kk = 0; kk < PK / 16; ++kk)
-                        ptx::mma_ss(acc, ptx::smem_desc_sw128(sa + kk * 32, 16, 1024),
-                                    ptx::smem_desc_sw128(sa + L::kA + kk * 32, 16, 1024), idesc,
-                                    (kb > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < PK / 16; ++kk) {
+                        const uint64_t bd = ptx::smem_desc_sw128(sa + L::kA + kk * 32, 16, 1024);
+                        const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+                        ptx::mma_ss(acc, ptx::smem_desc_sw128(sa + kk * 32, 16, 1024), bd, idesc, accum);
+                        ptx::mma_ss(acc + BN, ptx::smem_desc_sw128(sa + 128 * 128 + kk * 32, 16, 1024), bd,
+                                    idesc, accum);
+                    }
                     ptx::mma_commit(ctl.bar(L::bEmpty + s));
                 }
                 if (ok) ptx::mma_commit(ctl.bar(L::bAccFull + b));
@@ -286,49 +297,51 @@ projection_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
     } else {
         // ------------------------------------------------------------ epilogue
         const int qd = warp & 3;                      // TMEM lane quarter of this warp
-        const int row = qd * 32 + lane;
         int lt = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++lt) {
-            const int b = lt & 1;
-            if (!ctl.warp_wait(L::bAccFull + b, (lt >> 1) & 1) || *ctl.abort) break;
+            const int b = lt % L::kAccBuf;
+            if (!ctl.warp_wait(L::bAccFull + b, (lt / L::kAccBuf) & 1) || *ctl.abort) break;
             ptx::tc_fence_after();
             int mt, nt;
             tile_coords(tile, m_tiles, n_tiles, mt, nt);
             const int m0 = mt * PM, n0 = nt * BN;
-            const int r = m0 + row;
             const int seg_i = n0 / a.seg_w;
             const Seg& sg = a.seg[seg_i];
             const int col0 = n0 - seg_i * a.seg_w;    // first column of the tile in its segment
-            int dst_row = -1;
-            if (r < a.m) {
-                dst_row = sg.rowmap ? __ldg(sg.rowmap + r) : r;
-                if (dst_row < 0 || dst_row >= sg.n_rows) {
-                    raise_error(a.err, JANO_EINDEX);
-                    dst_row = -1;
-                }
-            }
-            const uint32_t taddr = tmem + b * BN + ((uint32_t)(qd * 32) << 16);
-            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(sg.dst) +
-                                  (size_t)(dst_row < 0 ? 0 : dst_row) * sg.ld + col0;
             const int cols = min(BN, a.seg_w - col0);  // columns of this tile inside the segment
 #pragma unroll 1
-            for (int cc = 0; cc < BN / 32; ++cc) {
-                uint32_t v[32];
-                ptx::tmem_ld32(taddr + 32 * cc, v);
-                ptx::tmem_wait_ld();
-                uint32_t pk[16];
+            for (int half = 0; half < 2; ++half) {
+                const int r = m0 + 128 * half + qd * 32 + lane;
+                int dst_row = -1;
+                if (r < a.m) {
+                    dst_row = sg.rowmap ? __ldg(sg.rowmap + r) : r;
+                    if (dst_row < 0 || dst_row >= sg.n_rows) {
+                        raise_error(a.err, JANO_EINDEX);
+                        dst_row = -1;
+                    }
+                }
+                const uint32_t taddr = tmem + (b * 2 + half) * BN + ((uint32_t)(qd * 32) << 16);
+                __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(sg.dst) +
+                                      (size_t)(dst_row < 0 ? 0 : dst_row) * sg.ld + col0;
+#pragma unroll 1
+                for (int cc = 0; cc < BN / 32; ++cc) {
+                    uint32_t v[32];
+                    ptx::tmem_ld32(taddr + 32 * cc, v);
+                    ptx::tmem_wait_ld();
+                    uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    pk[e] = ptx::pack_bf16(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-                if (dst_row >= 0) {
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = ptx::pack_bf16(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+                    if (dst_row >= 0) {
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        if (32 * cc + 8 * u < cols)
-                            *reinterpret_cast<uint4*>(orow + 32 * cc + 8 * u) =
-                                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                        for (int u = 0; u < 4; ++u)
+                            if (32 * cc + 8 * u < cols)
+                                *reinterpret_cast<uint4*>(orow + 32 * cc + 8 * u) =
+                                    make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                    }
                 }
             }
-            // this accumulator may take the next tile
+            // this accumulator set may take the next tile
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(ctl.bar(L::bAccEmpty + b));
@@ -338,7 +351,7 @@ projection_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, 2 * BN);
+    if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, 512);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
