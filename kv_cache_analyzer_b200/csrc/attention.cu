@@ -100,12 +100,17 @@ struct Ctl {
     __device__ uint32_t bar(int i) const { return bar0 + 8u * (uint32_t)i; }
     // Waiting threads are suspended (not spinning) until the phase completes,
     // leaving the issue slots to the softmax warps that share their
-    // sub-partition.
-    __device__ bool wait(int i, uint32_t parity) const {
-        if (ptx::mbar_try_wait_sleep(bar(i), parity)) return true;
+    // sub-partition; the MMA thread, whose waits for P and for K/V tiles sit
+    // on every key tile's critical path, polls instead (spin), which wakes
+    // it sooner.
+    __device__ bool wait(int i, uint32_t parity, bool spin = false) const {
+        auto poll = [&]() {
+            return spin ? ptx::mbar_try_wait(bar(i), parity) : ptx::mbar_try_wait_sleep(bar(i), parity);
+        };
+        if (poll()) return true;
         const long long t0 = clock64();
         for (;;) {
-            if (ptx::mbar_try_wait_sleep(bar(i), parity)) return true;
+            if (poll()) return true;
             if (*abort) return false;
             if (clock64() - t0 > kWaitLimit) {
                 *abort = 1;
@@ -355,7 +360,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
             constexpr uint32_t idesc_qk = ptx::idesc_bf16(BM, BN, false, false);
             constexpr uint32_t idesc_pv = ptx::idesc_bf16(BM, HD, false, true);
             auto slot_of = [](int n) { return n % kSlots; };
-            auto wait_full = [&](int n) { return ctl.wait(L::bFull + slot_of(n), (n / kSlots) & 1); };
+            auto wait_full = [&](int n) { return ctl.wait(L::bFull + slot_of(n), (n / kSlots) & 1, true); };
             auto qk = [&](int i, int n) {          // S_i = Q_i K^T, K in load n's slot
                 const uint32_t kb = base + L::kRing + slot_of(n) * L::kTile;
                 const uint32_t qb = base + (i ? L::kQ1 : L::kQ0);
@@ -377,10 +382,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
             };
             // P_i of tile j: upper key half as soon as it is published, then the lower half
             auto pv_tile = [&](int i, int n, int j) -> bool {
-                if (!ctl.wait(L::bPHalf + i, j & 1)) return false;
+                if (!ctl.wait(L::bPHalf + i, j & 1, true)) return false;
                 ptx::tc_fence_after();
                 pv(i, n, BN / 32, BN / 16, j > 0);
-                if (!ctl.wait(L::bPFull + i, j & 1)) return false;
+                if (!ctl.wait(L::bPFull + i, j & 1, true)) return false;
                 ptx::tc_fence_after();
                 pv(i, n, 0, BN / 32, true);
                 return true;
