@@ -302,7 +302,7 @@ def measure_attention_sizes(J, hp, stream, pk, reps=3):
     for name, (start, n) in cases.items():
         idx = hp.idx[start:start + n]
         qn = q[:n]
-        fn = lambda: J.jano_active_attention(qn, hp.k_cache, hp.v_cache, idx, n, N, H, d, d ** -0.5, out, stream)
+        fn = lambda: J.attention_auto(qn, hp.k_cache, hp.v_cache, idx, n, N, H, d, out, stream, hp.att_ws)
         fn()
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
         evs[0].record(stream)
@@ -538,7 +538,7 @@ def run_gpu(args, w, rank, world, local_rank, dist):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": cfg, "roofline": roofline, "cpu_baseline": cpu,
-            "e2e": e2e, "gpu_launches": KERNELS_PER_STEP * args.steps, "clocks": clk.summary(),
+            "e2e": e2e, "gpu_launches": (KERNELS_PER_STEP + (1 if hp.last_split > 1 else 0)) * args.steps, "clocks": clk.summary(),
             "kernels": kernels, "next_rows": next_rows,
             "peaks": {"source": pk_src, "hbm_gbs": hbm,
                                           "bf16_tflops": pk["bf16_tflops"],

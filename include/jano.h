@@ -245,6 +245,47 @@ JANO_API jano_status jano_active_attention(const void *q_act, const void *k_cach
                                   float scale, void *out, void *stream);
 
 /* ------------------------------------------------------------------------
+ * jano_active_attention_split -- jano_active_attention with each query
+ * tile's keys cut into n_split ranges, one CTA per range, for due sets too
+ * small to fill the GPU (same pages as jano_active_attention; splitting the
+ * keys is valid because the softmax denominator and the weighted sum of V
+ * are both sums over the keys).  Every range yields, per (query, head) row,
+ * its unnormalised output O_s (fp32), its running maximum m_s (log2 domain)
+ * and its sum l_s; a second pass merges them in split order:
+ *   out[idx[i], h] = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,
+ *   M = max_s m_s.
+ * Arguments as jano_active_attention, plus:
+ * n_split    1 .. ceil(n_tokens / 128); 1 behaves as jano_active_attention
+ *            (workspace unused).
+ * workspace  device buffer of ws_bytes >= jano_active_attention_workspace_bytes
+ *            (n_act, heads, d, n_split), 16-byte aligned, owned by the
+ *            caller; its contents are overwritten and need no zeroing.  The
+ *            calls that share it must be ordered on one stream.
+ * Errors: n_split out of range, or a NULL / too small workspace ->
+ * JANO_EINVAL; a misaligned workspace -> JANO_EALIGN; the rest as
+ * jano_active_attention.
+ * ---------------------------------------------------------------------- */
+JANO_API jano_status jano_active_attention_split(const void *q_act, const void *k_cache,
+                                        const void *v_cache, const int32_t *idx,
+                                        int n_act, int n_tokens, int heads, int d,
+                                        float scale, int n_split, void *workspace,
+                                        size_t ws_bytes, void *out, void *stream);
+
+/* Workspace bytes jano_active_attention_split needs (0 for n_split <= 1):
+ * n_split * n_act * heads * d fp32 partial rows, rounded up to 256 bytes,
+ * then n_split * n_act * heads (m, l) fp32 pairs. */
+JANO_API size_t jano_active_attention_workspace_bytes(int n_act, int heads, int d, int n_split);
+
+/* The key split that fills the current device's SMs best for this shape:
+ * with C = ceil(n_act / 256) * heads CTAs per split and S SMs, the split
+ * z (at most 16, at least 8 key tiles of 128 per CTA) that maximises
+ * w / ceil(w) * (1 - 0.02 (z - 1)), w = z C / S: the busy share of the
+ * last wave, less an allowance for the partials and the merge pass.
+ * Returns 1 when no split pays (call jano_active_attention then), or 1 on
+ * any error. */
+JANO_API int jano_active_attention_splits(int n_act, int n_tokens, int heads, int d);
+
+/* ------------------------------------------------------------------------
  * jano_gather_gemm -- a linear layer on the active rows only, rows gathered
  * on the way in and optionally scattered on the way out.  Pages: nl
  * technical summary, Methodologie 2 "KV Cache Mechanisme" (per step only a

@@ -23,6 +23,7 @@ __all__ = [
     "JanoError", "jano_geom", "jano_sched_cfg", "lib", "library_path",
     "jano_block_scores", "jano_classify", "jano_build_schedule_workspace_bytes",
     "jano_build_schedule", "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention",
+    "jano_active_attention_split", "jano_active_attention_workspace_bytes", "jano_active_attention_splits",
     "jano_get_device_error", "jano_status_str", "jano_version",
     "Geometry", "Schedule", "block_scores", "classify", "build_schedule",
     "kv_scatter", "active_attention", "device_error",
@@ -38,6 +39,7 @@ STATUS_NAMES = {0: "JANO_OK", 1: "JANO_EINVAL", 2: "JANO_ESHAPE", 3: "JANO_EALIG
                 7: "JANO_ETIMEOUT", 8: "JANO_ECUDA"}
 EXPORTS = ("jano_block_scores", "jano_block_scores_literal", "jano_classify", "jano_build_schedule_workspace_bytes",
            "jano_build_schedule", "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention",
+           "jano_active_attention_split", "jano_active_attention_workspace_bytes", "jano_active_attention_splits",
            "jano_gather_gemm", "jano_qkv_project", "jano_random_scores", "jano_fft_scores",
            "jano_get_device_error", "jano_status_str", "jano_version")
 
@@ -78,6 +80,11 @@ def lib() -> C.CDLL:
         L.jano_build_schedule_noalloc.argtypes = [P, G, S, P, P, z, P, P]
         L.jano_kv_scatter.argtypes = [P, P, P, i, i, i, P, P, i, P]
         L.jano_active_attention.argtypes = [P, P, P, P, i, i, i, i, f, P, P]
+        L.jano_active_attention_split.argtypes = [P, P, P, P, i, i, i, i, f, i, P, z, P, P]
+        L.jano_active_attention_workspace_bytes.argtypes = [i, i, i, i]
+        L.jano_active_attention_workspace_bytes.restype = z
+        L.jano_active_attention_splits.argtypes = [i, i, i, i]
+        L.jano_active_attention_splits.restype = C.c_int
         L.jano_gather_gemm.argtypes = [P, i, P, i, P, i, i, P, P, i, P]
         L.jano_qkv_project.argtypes = [P, i, P, i, P, i, i, P, P, P, P]
         L.jano_random_scores.argtypes = [i, C.c_uint64, P, P]
@@ -87,7 +94,8 @@ def lib() -> C.CDLL:
         L.jano_status_str.restype = C.c_char_p
         L.jano_version.argtypes = []
         for fn in ("jano_block_scores", "jano_block_scores_literal", "jano_classify", "jano_build_schedule",
-                   "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention", "jano_get_device_error",
+                   "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention",
+                   "jano_active_attention_split", "jano_get_device_error",
                    "jano_gather_gemm", "jano_qkv_project", "jano_random_scores", "jano_fft_scores",
                    "jano_version"):
             getattr(L, fn).restype = C.c_int
@@ -177,6 +185,23 @@ def jano_active_attention(q_act, k_cache, v_cache, idx, n_act, n_tokens, heads, 
         _dev(q_act, "q_act", torch.bfloat16), _dev(k_cache, "k_cache", torch.bfloat16),
         _dev(v_cache, "v_cache", torch.bfloat16), _dev(idx, "idx", torch.int32), n_act,
         n_tokens, heads, d, scale, _dev(out, "out", torch.bfloat16), _stream(stream)))
+
+
+def jano_active_attention_split(q_act, k_cache, v_cache, idx, n_act, n_tokens, heads, d, scale,
+                                n_split, workspace, ws_bytes, out, stream=None):
+    _check("jano_active_attention_split", lib().jano_active_attention_split(
+        _dev(q_act, "q_act", torch.bfloat16), _dev(k_cache, "k_cache", torch.bfloat16),
+        _dev(v_cache, "v_cache", torch.bfloat16), _dev(idx, "idx", torch.int32), n_act,
+        n_tokens, heads, d, scale, n_split, _dev(workspace, "workspace"), ws_bytes,
+        _dev(out, "out", torch.bfloat16), _stream(stream)))
+
+
+def jano_active_attention_workspace_bytes(n_act, heads, d, n_split) -> int:
+    return int(lib().jano_active_attention_workspace_bytes(n_act, heads, d, n_split))
+
+
+def jano_active_attention_splits(n_act, n_tokens, heads, d) -> int:
+    return int(lib().jano_active_attention_splits(n_act, n_tokens, heads, d))
 
 
 def jano_gather_gemm(x, n_x, gather, m, w, n, k, scatter, out, n_out, stream=None):
@@ -304,12 +329,57 @@ def kv_scatter(k_act, v_act, idx, k_cache, v_cache, stream=None) -> None:
     jano_kv_scatter(k_act, v_act, idx, n_act, H, d, k_cache, v_cache, N, stream)
 
 
-def active_attention(q_act, k_cache, v_cache, idx, out, scale=None, stream=None) -> None:
+def active_attention(q_act, k_cache, v_cache, idx, out, scale=None, stream=None, split=None,
+                     workspace=None) -> None:
+    """out[idx[i]] = attention of q_act[i] over the whole cache.  split: the
+    number of key ranges per query tile (None: the library's choice for this
+    shape on the current device, 1 for large due sets); with split > 1 the
+    partials go to `workspace` (a device uint8 tensor of at least
+    jano_active_attention_workspace_bytes bytes), allocated here if None."""
     n_act = idx.numel()
     N, H, d = k_cache.shape
     if scale is None:
         scale = d ** -0.5
-    jano_active_attention(q_act, k_cache, v_cache, idx, n_act, N, H, d, scale, out, stream)
+    if split is None:
+        split = jano_active_attention_splits(n_act, N, H, d) if n_act > 0 else 1
+    if split <= 1:
+        jano_active_attention(q_act, k_cache, v_cache, idx, n_act, N, H, d, scale, out, stream)
+        return
+    ws_bytes = jano_active_attention_workspace_bytes(n_act, H, d, split)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=k_cache.device)
+    jano_active_attention_split(q_act, k_cache, v_cache, idx, n_act, N, H, d, scale, split,
+                                workspace, workspace.numel() * workspace.element_size(), out, stream)
+
+
+class SplitWorkspace:
+    """Device workspace of key-split attention for one stream, grown on demand."""
+
+    def __init__(self, device):
+        self.device = torch.device(device)
+        self.buf = None
+
+    def get(self, nbytes: int, stream) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes:
+            with torch.cuda.stream(stream):
+                self.buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+def attention_auto(q_act, k_cache, v_cache, idx, n_act, n_tokens, heads, d, out, stream,
+                   ws: SplitWorkspace) -> int:
+    """jano_active_attention, or its key-split form when the library's choice
+    for this shape on this device is a split (small due sets, few heads);
+    returns the split count used."""
+    split = jano_active_attention_splits(n_act, n_tokens, heads, d) if n_act > 0 else 1
+    if split <= 1:
+        jano_active_attention(q_act, k_cache, v_cache, idx, n_act, n_tokens, heads, d, d ** -0.5,
+                              out, stream)
+        return 1
+    buf = ws.get(jano_active_attention_workspace_bytes(n_act, heads, d, split), stream)
+    jano_active_attention_split(q_act, k_cache, v_cache, idx, n_act, n_tokens, heads, d, d ** -0.5,
+                                split, buf, buf.numel(), out, stream)
+    return split
 
 
 def gather_gemm(x, w, out, gather=None, scatter=None, stream=None) -> None:

@@ -40,6 +40,7 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <cmath>
 #include <mutex>
 
 #include "jano_common.cuh"
@@ -269,13 +270,16 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, uint32_t 
     ptx::tmem_wait_st();
 }
 
-template <int HD>
+// kSplit: the key-split form (grid z = splits, partials to part_o / part_ml);
+// otherwise one CTA takes all keys and writes the normalised BF16 rows.
+template <int HD, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
 attention_kernel(const __grid_constant__ CUtensorMap tmQ,
                  const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV,
                  const int32_t* __restrict__ idx, int n_act, int n_tokens, int heads,
-                 float scale_log2, __nv_bfloat16* __restrict__ out, int* err) {
+                 float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ part_o,
+                 float2* __restrict__ part_ml, int* err) {
     using L = Layout<HD>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = ptx::smem_u32(smem_raw);
@@ -285,7 +289,12 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int head = blockIdx.y;
     const int q0 = blockIdx.x * 2 * BM;                // first query row of tile 0
-    const int nt = (n_tokens + BN - 1) / BN;
+    // key split: CTA z of n_split takes key tiles [kt0, kt1) of the nt_all
+    const int nt_all = (n_tokens + BN - 1) / BN;
+    const int n_split = kSplit ? (int)gridDim.z : 1, split = kSplit ? (int)blockIdx.z : 0;
+    const int kt0 = kSplit ? (int)((long long)nt_all * split / n_split) : 0;
+    const int kt1 = kSplit ? (int)((long long)nt_all * (split + 1) / n_split) : nt_all;
+    const int nt = kt1 - kt0;                          // key tiles of this CTA
 
     Ctl ctl;
     ctl.bar0 = base + L::kBar;
@@ -346,7 +355,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
                 const CUtensorMap* tm = (n & 1) ? &tmV : &tmK;
                 for (int p = 0; p < L::kPanels; ++p)
                     ptx::tma_load_3d(base + L::kRing + s * L::kTile + p * kPanel, tm,
-                                     ctl.bar(L::bFull + s), p * 64, head, (n >> 1) * BN);
+                                     ctl.bar(L::bFull + s), p * 64, head, (kt0 + (n >> 1)) * BN);
                 last[s] = n;
             }
             // drain: every copy this CTA issued lands before its smem is released
@@ -447,7 +456,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
         }
         float m = -INFINITY, l = 0.f;
-        const int tail = n_tokens - (nt - 1) * BN;    // valid keys in the last tile
+        // valid keys in this CTA's last tile (only the sequence's last tile is ragged)
+        const int tail = kt1 == nt_all ? n_tokens - (nt_all - 1) * BN : BN;
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
             if (!ctl.warp_wait(L::bSFull + i, j & 1)) { ok = false; break; }
@@ -463,23 +473,44 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         // ------------------------------------------------------------ epilogue
         if (ok && ctl.warp_wait(L::bOFull + i, 0)) {
             ptx::tc_fence_after();
-            const float inv = 1.0f / l;
-            __nv_bfloat16* orow = out + ((size_t)(t_out < 0 ? 0 : t_out) * heads + head) * HD;
+            if constexpr (!kSplit) {
+                const float inv = 1.0f / l;
+                __nv_bfloat16* orow = out + ((size_t)(t_out < 0 ? 0 : t_out) * heads + head) * HD;
 #pragma unroll
-            for (int c = 0; c < HD / 32; ++c) {
-                uint32_t o[32];
-                ptx::tmem_ld32(tO + 32 * c, o);
-                ptx::tmem_wait_ld();
-                uint32_t pk[16];
+                for (int c = 0; c < HD / 32; ++c) {
+                    uint32_t o[32];
+                    ptx::tmem_ld32(tO + 32 * c, o);
+                    ptx::tmem_wait_ld();
+                    uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    pk[e] = ptx::pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-                if (t_out >= 0) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = ptx::pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+                    if (t_out >= 0) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                        for (int v = 0; v < 4; ++v)
+                            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    }
                 }
+            } else {
+                // key split: this CTA's unnormalised O (fp32) with its row max m
+                // (log2 domain) and sum l, for the combine pass
+                const bool live = qi < n_act;
+                const size_t prow = ((size_t)split * n_act + (live ? qi : 0)) * heads + head;
+                float4* po = reinterpret_cast<float4*>(part_o + prow * HD);
+#pragma unroll
+                for (int c = 0; c < HD / 32; ++c) {
+                    uint32_t o[32];
+                    ptx::tmem_ld32(tO + 32 * c, o);
+                    ptx::tmem_wait_ld();
+                    if (live) {
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            po[8 * c + v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                                        __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+                    }
+                }
+                if (live) part_ml[prow] = make_float2(m, l);
             }
         }
     }
@@ -488,6 +519,57 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
     __syncthreads();
     ptx::tc_fence_after();
     if (warp == 9) ptx::tmem_dealloc(tmem, 512);
+}
+
+// Merge of the key-split partials: one warp per (query, head) row; lane
+// holds HD/32 consecutive columns.  With M = max_s m_s and w_s = 2^(m_s - M),
+//   out[idx[i], h] = sum_s w_s O_s / sum_s w_s l_s,
+// summed over the splits in order (deterministic).
+template <int HD>
+__global__ void __launch_bounds__(256)
+attention_combine_kernel(const float* __restrict__ part_o, const float2* __restrict__ part_ml,
+                         const int32_t* __restrict__ idx, int n_act, int n_tokens, int heads,
+                         int n_split, __nv_bfloat16* __restrict__ out, int* err) {
+    constexpr int E = HD / 32;
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const long long rows = (long long)n_act * heads;
+    if (row >= rows) return;
+    const int qi = (int)(row / heads), head = (int)(row % heads);
+    const int t = __ldg(idx + qi);
+    if (t < 0 || t >= n_tokens) {
+        if (lane == 0) raise_error(err, JANO_EINDEX);
+        return;
+    }
+    float M = -INFINITY;
+    for (int z = 0; z < n_split; ++z) M = fmaxf(M, part_ml[z * rows + row].x);
+    float acc[E], L = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    for (int z = 0; z < n_split; ++z) {
+        const float2 ml = part_ml[z * rows + row];
+        const float w = ptx::ex2(ml.x - M);
+        L = fmaf(w, ml.y, L);
+        const float* src = part_o + (z * rows + row) * HD + lane * E;
+        float v[E];
+        if constexpr (E == 4) {
+            const float4 x = *reinterpret_cast<const float4*>(src);
+            v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+        } else {
+            const float2 x = *reinterpret_cast<const float2*>(src);
+            v[0] = x.x; v[1] = x.y;
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = fmaf(w, v[e], acc[e]);
+    }
+    const float inv = 1.0f / L;
+    __nv_bfloat16* dst = out + ((size_t)t * heads + head) * HD + lane * E;
+    if constexpr (E == 4) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(ptx::pack_bf16(acc[0] * inv, acc[1] * inv),
+                                                    ptx::pack_bf16(acc[2] * inv, acc[3] * inv));
+    } else {
+        *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16(acc[0] * inv, acc[1] * inv);
+    }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -516,10 +598,10 @@ bool make_map(CUtensorMap* m, const void* ptr, int rows, int heads, int d) {
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int HD>
+template <int HD, bool kSplit>
 cudaError_t launch_hd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const int32_t* idx, int n_act, int n_tokens, int heads, float scale,
-                      void* out, int* err, cudaStream_t st) {
+                      void* out, int n_split, void* ws, int* err, cudaStream_t st) {
     using L = Layout<HD>;
     // the shared-memory opt-in is per device: remember which devices have it
     static DeviceOnce ready;
@@ -529,36 +611,88 @@ cudaError_t launch_hd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
         // the register split assumes exactly kRegsLaunch registers per thread
         // at launch; anything else could leave an increase waiting for good
         cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, attention_kernel<HD>);
+        cudaError_t e = cudaFuncGetAttributes(&fa, attention_kernel<HD, kSplit>);
         if (e != cudaSuccess) return e;
         if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(attention_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(attention_kernel<HD, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)L::kAlloc);
         if (e != cudaSuccess) return e;
         ready.mark(dev);
     }
     const int q_tiles = (n_act + BM - 1) / BM;
-    const dim3 grid((q_tiles + 1) / 2, heads);
+    const dim3 grid((q_tiles + 1) / 2, heads, n_split);
     const float scale_log2 = scale * 1.4426950408889634f;
-    attention_kernel<HD><<<grid, kThreads, L::kAlloc, st>>>(
+    float* part_o = nullptr;
+    float2* part_ml = nullptr;
+    if (kSplit) {
+        part_o = static_cast<float*>(ws);
+        part_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) +
+                                            attention_partials_bytes(n_act, heads, HD, n_split));
+    }
+    attention_kernel<HD, kSplit><<<grid, kThreads, L::kAlloc, st>>>(
         mq, mk, mv, idx, n_act, n_tokens, heads, scale_log2,
-        static_cast<__nv_bfloat16*>(out), err);
+        static_cast<__nv_bfloat16*>(out), part_o, part_ml, err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || !kSplit) return e;
+    const long long rows = (long long)n_act * heads;
+    attention_combine_kernel<HD><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+        part_o, part_ml, idx, n_act, n_tokens, heads, n_split, static_cast<__nv_bfloat16*>(out), err);
     return cudaGetLastError();
 }
 
 }  // namespace
 
+size_t attention_partials_bytes(int n_act, int heads, int d, int n_split) {
+    const size_t o = (size_t)n_split * n_act * heads * d * sizeof(float);
+    return (o + 255) / 256 * 256;
+}
+
+size_t attention_workspace_bytes(int n_act, int heads, int d, int n_split) {
+    if (n_split <= 1) return 0;
+    return attention_partials_bytes(n_act, heads, d, n_split) + (size_t)n_split * n_act * heads * 8;
+}
+
+int attention_key_tiles(int n_tokens) { return (n_tokens + BN - 1) / BN; }
+
+// Key splits that fill the SMs best: the fraction of the last wave that is
+// busy (waves / ceil(waves)), less 2% per extra split for the partials'
+// round trip and the combine pass; at least 8 key tiles per CTA.
+int attention_split_count(int n_act, int n_tokens, int heads, int sms) {
+    if (n_act <= 0 || sms <= 0) return 1;
+    const long long ctas = (long long)((n_act + 2 * BM - 1) / (2 * BM)) * heads;
+    const int nt = attention_key_tiles(n_tokens);
+    int best = 1;
+    double best_score = 0.0;
+    for (int z = 1; z <= 16 && nt / z >= 8; ++z) {
+        const double waves = (double)(ctas * z) / sms;
+        const double score = waves / std::ceil(waves) * (1.0 - 0.02 * (z - 1));
+        if (score > best_score + 1e-9) {
+            best_score = score;
+            best = z;
+        }
+    }
+    return best;
+}
+
 cudaError_t launch_active_attention(const void* q, const void* k, const void* v,
                                     const int32_t* idx, int n_act, int n_tokens,
                                     int heads, int d, float scale, void* out,
-                                    int* err, cudaStream_t st) {
+                                    int* err, cudaStream_t st, int n_split, void* ws) {
     if (n_act <= 0) return cudaSuccess;
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, n_act, heads, d) || !make_map(&mk, k, n_tokens, heads, d) ||
         !make_map(&mv, v, n_tokens, heads, d))
         return cudaErrorInvalidValue;
-    if (d == 128) return launch_hd<128>(mq, mk, mv, idx, n_act, n_tokens, heads, scale, out, err, st);
-    return launch_hd<64>(mq, mk, mv, idx, n_act, n_tokens, heads, scale, out, err, st);
+    if (n_split < 1 || n_split > attention_key_tiles(n_tokens) || (n_split > 1 && !ws))
+        return cudaErrorInvalidValue;
+    if (n_split > 1) {
+        if (d == 128)
+            return launch_hd<128, true>(mq, mk, mv, idx, n_act, n_tokens, heads, scale, out, n_split, ws, err, st);
+        return launch_hd<64, true>(mq, mk, mv, idx, n_act, n_tokens, heads, scale, out, n_split, ws, err, st);
+    }
+    if (d == 128)
+        return launch_hd<128, false>(mq, mk, mv, idx, n_act, n_tokens, heads, scale, out, 1, nullptr, err, st);
+    return launch_hd<64, false>(mq, mk, mv, idx, n_act, n_tokens, heads, scale, out, 1, nullptr, err, st);
 }
 
 }  // namespace jano

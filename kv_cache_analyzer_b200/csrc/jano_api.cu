@@ -163,6 +163,45 @@ jano_status jano_active_attention(const void* q_act, const void* k_cache, const 
                                              d, scale, out, err, static_cast<cudaStream_t>(stream)));
 }
 
+jano_status jano_active_attention_split(const void* q_act, const void* k_cache, const void* v_cache,
+                                        const int32_t* idx, int n_act, int n_tokens, int heads, int d,
+                                        float scale, int n_split, void* workspace, size_t ws_bytes,
+                                        void* out, void* stream) {
+    if (n_act < 0 || n_tokens < 1 || heads < 1) return JANO_EINVAL;
+    if (!(scale > 0.0f) || !std::isfinite(scale)) return JANO_EINVAL;
+    if (d != 64 && d != 128) return JANO_EUNSUPPORTED;
+    if (heads > 65535) return JANO_EUNSUPPORTED;
+    if (n_split < 1 || n_split > attention_key_tiles(n_tokens)) return JANO_EINVAL;
+    if (n_split == 1)
+        return jano_active_attention(q_act, k_cache, v_cache, idx, n_act, n_tokens, heads, d, scale,
+                                     out, stream);
+    if (n_act == 0) return JANO_OK;
+    if (!workspace || ws_bytes < attention_workspace_bytes(n_act, heads, d, n_split)) return JANO_EINVAL;
+    if (!aligned16(workspace)) return JANO_EALIGN;
+    if (!q_act || !k_cache || !v_cache || !idx || !out) return JANO_EINVAL;
+    if (!aligned16(q_act) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return JANO_EALIGN;
+    int* err = device_error_word();
+    if (!err) return JANO_ECUDA;
+    return from_cuda(launch_active_attention(q_act, k_cache, v_cache, idx, n_act, n_tokens, heads, d,
+                                             scale, out, err, static_cast<cudaStream_t>(stream),
+                                             n_split, workspace));
+}
+
+size_t jano_active_attention_workspace_bytes(int n_act, int heads, int d, int n_split) {
+    if (n_act <= 0 || heads <= 0 || d <= 0 || n_split <= 1) return 0;
+    return attention_workspace_bytes(n_act, heads, d, n_split);
+}
+
+int jano_active_attention_splits(int n_act, int n_tokens, int heads, int d) {
+    if (n_act <= 0 || n_tokens < 1 || heads < 1 || (d != 64 && d != 128)) return 1;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 1;
+    return attention_split_count(n_act, n_tokens, heads, sms);
+}
+
 jano_status jano_gather_gemm(const void* x, int n_x, const int32_t* gather, int m, const void* w,
                              int n, int k, const int32_t* scatter, void* out, int n_out,
                              void* stream) {

@@ -61,10 +61,17 @@ cudaError_t launch_build_schedule(const uint8_t* block_levels, const jano_geom& 
 cudaError_t launch_kv_scatter(const void* k_act, const void* v_act, const int32_t* idx,
                               int n_act, int row_bytes, void* k_cache, void* v_cache,
                               int n_tokens, int* err, cudaStream_t st);
+// n_split > 1: each query tile's keys are cut into n_split ranges, one CTA
+// each, whose partials go to ws (attention_workspace_bytes) and are merged
+// by a combine pass.
 cudaError_t launch_active_attention(const void* q, const void* k, const void* v,
                                     const int32_t* idx, int n_act, int n_tokens,
                                     int heads, int d, float scale, void* out,
-                                    int* err, cudaStream_t st);
+                                    int* err, cudaStream_t st, int n_split = 1, void* ws = nullptr);
+size_t attention_partials_bytes(int n_act, int heads, int d, int n_split);
+size_t attention_workspace_bytes(int n_act, int heads, int d, int n_split);
+int attention_key_tiles(int n_tokens);
+int attention_split_count(int n_act, int n_tokens, int heads, int sms);
 
 // One output segment of the projection kernel: its columns go to `dst`
 // (BF16 rows of `ld` elements) at row rowmap[r] (or r when rowmap is NULL).

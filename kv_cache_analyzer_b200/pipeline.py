@@ -9,6 +9,7 @@ sampling step of the method:
   a3  jano_build_schedule   token levels        -> per-step due lists (CSR)
   a4  jano_kv_scatter       fresh K/V of the due tokens -> persistent cache
   a5  jano_active_attention due queries over the whole cache -> out[idx]
+      (jano_active_attention_split for due sets too small to fill the GPU)
 
 The CSR offsets are read back to the host once by ``plan()`` (one small
 device-to-host copy per generation); ``step(s)`` then runs a1..a5 for
@@ -20,11 +21,12 @@ from __future__ import annotations
 
 import torch
 
-from . import (Geometry, Schedule, jano_active_attention, jano_block_scores,
+from . import (Geometry, Schedule, SplitWorkspace, attention_auto, jano_block_scores,
                jano_build_schedule, jano_build_schedule_workspace_bytes,
                jano_classify, jano_kv_scatter)
 
 KERNELS_PER_STEP = 7      # scores 1 + classify 1 + schedule 3 + scatter 1 + attention 1
+                          # (attention 2 when its keys are split: + the merge pass)
 
 
 class HotPath:
@@ -54,6 +56,8 @@ class HotPath:
         self.k_cache = torch.empty((N, heads, d), dtype=torch.bfloat16, **e)
         self.v_cache = torch.empty((N, heads, d), dtype=torch.bfloat16, **e)
         self.out = torch.zeros((N, heads, d), dtype=torch.bfloat16, **e)
+        self.att_ws = SplitWorkspace(self.dev)   # key-split attention workspace
+        self.last_split = 1
         self.q_act = self.k_act = self.v_act = None
         self.host_offsets = None
         self._lgc, self._tgc, self._sc = lg.c(), token_geom.c(), sched.c()
@@ -108,8 +112,8 @@ class HotPath:
         jano_kv_scatter(self.k_act, self.v_act, idx, n_act, self.heads, self.d,
                         self.k_cache, self.v_cache, self.N, s)
         if ev[4] is not None: ev[4].record(s)
-        jano_active_attention(self.q_act, self.k_cache, self.v_cache, idx, n_act, self.N,
-                              self.heads, self.d, self.d ** -0.5, self.out, s)
+        self.last_split = attention_auto(self.q_act, self.k_cache, self.v_cache, idx, n_act, self.N,
+                                         self.heads, self.d, self.out, s, self.att_ws)
         if ev[5] is not None: ev[5].record(s)
         return n_act
 

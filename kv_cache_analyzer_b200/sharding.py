@@ -23,7 +23,7 @@ from typing import Callable, Optional
 
 import torch
 
-from . import (Geometry, Schedule, jano_active_attention, jano_block_scores,
+from . import (Geometry, Schedule, SplitWorkspace, attention_auto, jano_block_scores,
                jano_build_schedule, jano_build_schedule_workspace_bytes, jano_classify,
                jano_kv_scatter)
 
@@ -119,6 +119,8 @@ class ShardedHotPath:
         self.k_cache = torch.empty(shape, dtype=torch.bfloat16, **e)
         self.v_cache = torch.empty(shape, dtype=torch.bfloat16, **e)
         self.out = torch.zeros(shape, dtype=torch.bfloat16, **e)
+        self.att_ws = SplitWorkspace(self.dev)   # key-split attention workspace
+        self.last_split = 1
         self.q_act = self.k_act = self.v_act = None
         self.host_offsets = None
         self._sgc, self._tgc, self._sc = self.slab_geom.c(), token_geom.c(), sched.c()
@@ -182,8 +184,9 @@ class ShardedHotPath:
         idx = self.idx[start:start + n_act]
         jano_kv_scatter(self.k_act, self.v_act, idx, n_act, self.heads, self.d,
                         self.k_cache, self.v_cache, self.N, s)
-        jano_active_attention(self.q_act, self.k_cache, self.v_cache, idx, n_act, self.N,
-                              self.heads, self.d, self.d ** -0.5, self.out, s)
+        # a rank's few heads give few CTAs: the keys are split when that fills the SMs better
+        self.last_split = attention_auto(self.q_act, self.k_cache, self.v_cache, idx, n_act, self.N,
+                                         self.heads, self.d, self.out, s, self.att_ws)
         return n_act
 
     def run_step_kernels(self, step: int):

@@ -101,6 +101,34 @@ def test_host_validation_rejects_before_any_launch(jl):
     assert L.jano_fft_scores(nil, 16, C.byref(g4), 1, fake, nil) == 1
     g5 = jl.Geometry(4, 32, 32, (4, 8, 16), (1, 2, 2)).c()
     assert L.jano_fft_scores(fake, 16, C.byref(g5), 1, fake, nil) == 4
+    # key-split attention: split count out of range (0; more splits than
+    # key tiles of 128), NULL / short / misaligned workspace, an empty call
+    need = L.jano_active_attention_workspace_bytes(300, 4, 128, 3)
+    assert L.jano_active_attention_split(fake, fake, fake, fake, 300, 1024, 4, 128, 0.1, 0, fake,
+                                         need, fake, nil) == 1
+    assert L.jano_active_attention_split(fake, fake, fake, fake, 300, 1024, 4, 128, 0.1, 9, fake,
+                                         10**9, fake, nil) == 1
+    assert L.jano_active_attention_split(fake, fake, fake, fake, 300, 1024, 4, 128, 0.1, 3, nil,
+                                         need, fake, nil) == 1
+    assert L.jano_active_attention_split(fake, fake, fake, fake, 300, 1024, 4, 128, 0.1, 3, fake,
+                                         need - 1, fake, nil) == 1
+    assert L.jano_active_attention_split(fake, fake, fake, fake, 300, 1024, 4, 128, 0.1, 3,
+                                         C.c_void_p(264), need, fake, nil) == 3
+    assert L.jano_active_attention_split(nil, nil, nil, nil, 0, 1024, 4, 128, 0.1, 3, nil, 0,
+                                         nil, nil) == 0
+    assert L.jano_active_attention_split(fake, fake, fake, fake, 300, 1024, 4, 96, 0.1, 3, fake,
+                                         need, fake, nil) == 4
+
+
+def test_split_attention_workspace_and_choice_are_host_only(jl):
+    # n_split rows of fp32 partials (256-byte rounded), then (m, l) pairs
+    assert jl.jano_active_attention_workspace_bytes(300, 4, 128, 3) == 3 * 300 * 4 * 128 * 4 + 3 * 300 * 4 * 8
+    assert jl.jano_active_attention_workspace_bytes(5, 3, 64, 2) == 7680 + 2 * 5 * 3 * 8
+    assert jl.jano_active_attention_workspace_bytes(300, 4, 128, 1) == 0
+    assert jl.jano_active_attention_workspace_bytes(0, 4, 128, 3) == 0
+    # without a device the library recommends no split
+    if not __import__("torch").cuda.is_available():
+        assert jl.jano_active_attention_splits(3276, 32760, 12, 128) == 1
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch, jl):

@@ -94,5 +94,18 @@ def test_sharded_step_equals_unsharded(name, world):
         assert torch.equal(_bits(sh.scores), s_ref), f"rank {sh.rank} scores"
         assert torch.equal(sh.offsets.cpu(), off_ref)
         assert torch.equal(sh.idx[:n_due].cpu(), idx_ref)
-        for mine, theirs in ((sh.k_cache, ref.k_cache), (sh.v_cache, ref.v_cache), (sh.out, ref.out)):
+        for mine, theirs in ((sh.k_cache, ref.k_cache), (sh.v_cache, ref.v_cache)):
             assert torch.equal(_bits(mine), _bits(sh.head_slice(theirs))), f"rank {sh.rank} heads"
+        if sh.heads == 0:
+            continue
+        if sh.last_split == ref.last_split:
+            assert torch.equal(_bits(sh.out), _bits(sh.head_slice(ref.out))), f"rank {sh.rank} out"
+        else:
+            # a rank with fewer heads has fewer CTAs and may split the keys where
+            # the whole step did not: the same attention up to the rounding of P
+            # and of the output to BF16, so the two agree within the attention
+            # tolerance (max-abs 2e-2, mean-rel 5e-3)
+            a = sh.head_slice(ref.out).float()
+            b = sh.out.float()
+            assert float((a - b).abs().max()) <= 2e-2, f"rank {sh.rank} out"
+            assert float((a - b).abs().sum() / a.abs().sum()) <= 5e-3, f"rank {sh.rank} out"
