@@ -276,13 +276,13 @@ JANO_API jano_status jano_active_attention_split(const void *q_act, const void *
  * then n_split * n_act * heads (m, l) fp32 pairs. */
 JANO_API size_t jano_active_attention_workspace_bytes(int n_act, int heads, int d, int n_split);
 
-/* The key split that fills the current device's SMs best for this shape:
- * with C = ceil(n_act / 256) * heads CTAs per split and S SMs, the split
- * z (at most 16, at least 8 key tiles of 128 per CTA) that maximises
- * w / ceil(w) * (1 - 0.02 (z - 1)), w = z C / S: the busy share of the
- * last wave, less an allowance for the partials and the merge pass.
- * Returns 1 when no split pays (call jano_active_attention then), or 1 on
- * any error. */
+/* The key split with the shortest modelled time on the current device: with
+ * C = ceil(n_act / 256) * heads CTAs per split, S SMs and nt = ceil(n_tokens
+ * / 128) key tiles, the z (at most 16, at least 8 key tiles per CTA) that
+ * minimises R(z) * (nt / z + 12), where R(z) counts floor(w) full rounds of
+ * w = z C / S and a partial last round of fraction f as 0.7 + 0.3 f (the
+ * constants are fitted to measured B200 sweeps).  Returns 1 when no split
+ * pays (call jano_active_attention then), or 1 on any error. */
 JANO_API int jano_active_attention_splits(int n_act, int n_tokens, int heads, int d);
 
 /* ------------------------------------------------------------------------

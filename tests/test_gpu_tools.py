@@ -39,3 +39,15 @@ def test_sharding_run(capsys):
         assert sum(p["frames"] for p in d["per_rank"]) == 3
         assert d["n_active"] == lines[0]["n_active"] > 0
     torch.cuda.synchronize()
+
+
+def test_split_run(capsys):
+    from kv_cache_analyzer_b200 import split_run
+    split_run.main(["--case", "2048", "2", "300", "--case", "300", "1", "40", "--splits", "1", "2", "3", "5",
+                    "--reps", "2"])
+    lines = _lines(capsys)
+    assert [d["n_act"] for d in lines] == [300, 40]
+    assert set(lines[0]["TFLOP/s"]) == {"1", "2", "3", "5"} and lines[0]["chosen"] >= 1
+    assert set(lines[1]["TFLOP/s"]) == {"1", "2", "3"}     # 3 key tiles: at most 3 ranges
+    assert lines[1]["chosen"] == 1                          # under 8 key tiles per range: no split
+    assert all(v > 0 for d in lines for v in d["TFLOP/s"].values())
