@@ -285,6 +285,10 @@ JANO_API size_t jano_active_attention_workspace_bytes(int n_act, int heads, int 
  * pays (call jano_active_attention then), or 1 on any error. */
 JANO_API int jano_active_attention_splits(int n_act, int n_tokens, int heads, int d);
 
+/* The same choice for a device of sm_count SMs (host only, no device
+ * query); 1 on invalid arguments. */
+JANO_API int jano_active_attention_splits_on(int n_act, int n_tokens, int heads, int d, int sm_count);
+
 /* ------------------------------------------------------------------------
  * jano_gather_gemm -- a linear layer on the active rows only, rows gathered
  * on the way in and optionally scattered on the way out.  Pages: nl

@@ -24,7 +24,7 @@ __all__ = [
     "jano_block_scores", "jano_classify", "jano_build_schedule_workspace_bytes",
     "jano_build_schedule", "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention",
     "jano_active_attention_split", "jano_active_attention_workspace_bytes", "jano_active_attention_splits",
-    "jano_get_device_error", "jano_status_str", "jano_version",
+    "jano_active_attention_splits_on", "jano_get_device_error", "jano_status_str", "jano_version",
     "Geometry", "Schedule", "block_scores", "classify", "build_schedule",
     "kv_scatter", "active_attention", "device_error",
 ]
@@ -40,7 +40,7 @@ STATUS_NAMES = {0: "JANO_OK", 1: "JANO_EINVAL", 2: "JANO_ESHAPE", 3: "JANO_EALIG
 EXPORTS = ("jano_block_scores", "jano_block_scores_literal", "jano_classify", "jano_build_schedule_workspace_bytes",
            "jano_build_schedule", "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention",
            "jano_active_attention_split", "jano_active_attention_workspace_bytes", "jano_active_attention_splits",
-           "jano_gather_gemm", "jano_qkv_project", "jano_random_scores", "jano_fft_scores",
+           "jano_active_attention_splits_on", "jano_gather_gemm", "jano_qkv_project", "jano_random_scores", "jano_fft_scores",
            "jano_get_device_error", "jano_status_str", "jano_version")
 
 
@@ -85,6 +85,8 @@ def lib() -> C.CDLL:
         L.jano_active_attention_workspace_bytes.restype = z
         L.jano_active_attention_splits.argtypes = [i, i, i, i]
         L.jano_active_attention_splits.restype = C.c_int
+        L.jano_active_attention_splits_on.argtypes = [i, i, i, i, i]
+        L.jano_active_attention_splits_on.restype = C.c_int
         L.jano_gather_gemm.argtypes = [P, i, P, i, P, i, i, P, P, i, P]
         L.jano_qkv_project.argtypes = [P, i, P, i, P, i, i, P, P, P, P]
         L.jano_random_scores.argtypes = [i, C.c_uint64, P, P]
@@ -202,6 +204,10 @@ def jano_active_attention_workspace_bytes(n_act, heads, d, n_split) -> int:
 
 def jano_active_attention_splits(n_act, n_tokens, heads, d) -> int:
     return int(lib().jano_active_attention_splits(n_act, n_tokens, heads, d))
+
+
+def jano_active_attention_splits_on(n_act, n_tokens, heads, d, sm_count) -> int:
+    return int(lib().jano_active_attention_splits_on(n_act, n_tokens, heads, d, sm_count))
 
 
 def jano_gather_gemm(x, n_x, gather, m, w, n, k, scatter, out, n_out, stream=None):

@@ -193,13 +193,17 @@ size_t jano_active_attention_workspace_bytes(int n_act, int heads, int d, int n_
     return attention_workspace_bytes(n_act, heads, d, n_split);
 }
 
+int jano_active_attention_splits_on(int n_act, int n_tokens, int heads, int d, int sm_count) {
+    if (n_act <= 0 || n_tokens < 1 || heads < 1 || (d != 64 && d != 128) || sm_count < 1) return 1;
+    return attention_split_count(n_act, n_tokens, heads, sm_count);
+}
+
 int jano_active_attention_splits(int n_act, int n_tokens, int heads, int d) {
-    if (n_act <= 0 || n_tokens < 1 || heads < 1 || (d != 64 && d != 128)) return 1;
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return 1;
-    return attention_split_count(n_act, n_tokens, heads, sms);
+    return jano_active_attention_splits_on(n_act, n_tokens, heads, d, sms);
 }
 
 jano_status jano_gather_gemm(const void* x, int n_x, const int32_t* gather, int m, const void* w,

@@ -155,3 +155,25 @@ def test_every_workload_geometry_passes_host_support_checks(jl):
         K1, Cc, F, H, W = shape
         g = jl.Geometry(F, H, W, block, (1, 1, 1)).c()
         assert L.jano_block_scores(fake, K1 - 1, Cc, C.byref(g), 0.5, 0.5, fake, None) != 4, shape
+
+
+def test_split_choice_on_a_given_sm_count(jl):
+    f = jl.jano_active_attention_splits_on
+    # the shapes of the measured split sweep, 148 SMs (B200)
+    assert [f(n, 32760, 12, 128, 148) for n in (1638, 3276, 8190, 16380, 24570, 32760)] == [3, 4, 1, 2, 1, 1]
+    assert f(18900, 75600, 5, 128, 148) == 2        # a rank of the 8-way head-sharded step
+    assert f(18900, 75600, 40, 128, 148) == 1       # the large step's due sets never split
+    assert f(41580, 75600, 40, 128, 148) == 1
+    assert f(75600, 75600, 40, 128, 148) == 1
+    # fewer than 16 key tiles: no range of 8+ tiles to split into
+    assert f(100, 1000, 1, 128, 148) == 1
+    assert f(1, 2049, 1, 64, 148) == 2              # 17 tiles: two ranges of 8+
+    # invalid arguments
+    assert f(100, 32760, 12, 96, 148) == 1
+    assert f(100, 32760, 12, 128, 0) == 1
+    assert f(0, 32760, 12, 128, 148) == 1
+    for sms in (1, 16, 148, 1000):
+        for n in (1, 300, 3276, 40000):
+            for N in (128, 1024, 32760, 75600):
+                z = f(n, N, 4, 128, sms)
+                assert 1 <= z <= 16 and (z == 1 or ((N + 127) // 128) // z >= 8)
