@@ -255,7 +255,7 @@ JANO_API jano_status jano_active_attention(const void *q_act, const void *k_cach
  *   out[idx[i], h] = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,
  *   M = max_s m_s.
  * Arguments as jano_active_attention, plus:
- * n_split    1 .. ceil(n_tokens / 128); 1 behaves as jano_active_attention
+ * n_split    1 .. min(ceil(n_tokens / 128), 65535); 1 behaves as jano_active_attention
  *            (workspace unused).
  * workspace  device buffer of ws_bytes >= jano_active_attention_workspace_bytes
  *            (n_act, heads, d, n_split), 16-byte aligned, owned by the

@@ -171,7 +171,7 @@ jano_status jano_active_attention_split(const void* q_act, const void* k_cache, 
     if (!(scale > 0.0f) || !std::isfinite(scale)) return JANO_EINVAL;
     if (d != 64 && d != 128) return JANO_EUNSUPPORTED;
     if (heads > 65535) return JANO_EUNSUPPORTED;
-    if (n_split < 1 || n_split > attention_key_tiles(n_tokens)) return JANO_EINVAL;
+    if (n_split < 1 || n_split > attention_key_tiles(n_tokens) || n_split > 65535) return JANO_EINVAL;
     if (n_split == 1)
         return jano_active_attention(q_act, k_cache, v_cache, idx, n_act, n_tokens, heads, d, scale,
                                      out, stream);
