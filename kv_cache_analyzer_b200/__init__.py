@@ -105,6 +105,16 @@ def lib() -> C.CDLL:
     return _lib
 
 
+def _torch_stream(stream):
+    """The torch stream object for `stream` (None: the current stream; a raw
+    cudaStream_t handle is wrapped), for allocator bookkeeping."""
+    if stream is None:
+        return torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return stream
+    return torch.cuda.ExternalStream(int(stream))
+
+
 def _stream(stream) -> C.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -352,10 +362,15 @@ def active_attention(q_act, k_cache, v_cache, idx, out, scale=None, stream=None,
         jano_active_attention(q_act, k_cache, v_cache, idx, n_act, N, H, d, scale, out, stream)
         return
     ws_bytes = jano_active_attention_workspace_bytes(n_act, H, d, split)
-    if workspace is None:
+    temporary = workspace is None
+    if temporary:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=k_cache.device)
     jano_active_attention_split(q_act, k_cache, v_cache, idx, n_act, N, H, d, scale, split,
                                 workspace, workspace.numel() * workspace.element_size(), out, stream)
+    if temporary:
+        # freed on return: the allocator must not hand it out again before the
+        # launch on `stream` has finished with it
+        workspace.record_stream(_torch_stream(stream))
 
 
 class SplitWorkspace:
@@ -367,7 +382,7 @@ class SplitWorkspace:
 
     def get(self, nbytes: int, stream) -> torch.Tensor:
         if self.buf is None or self.buf.numel() < nbytes:
-            with torch.cuda.stream(stream):
+            with torch.cuda.stream(_torch_stream(stream)):
                 self.buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         return self.buf
 
