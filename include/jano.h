@@ -11,7 +11,9 @@
  *   2. the per-step partial-token attention: fresh K/V of the due tokens are
  *      scattered into a persistent full-sequence cache (jano_kv_scatter) and
  *      only the due (active) queries attend over the whole cache
- *      (jano_active_attention), their outputs going back to their token rows.
+ *      (jano_active_attention, or jano_active_attention_split for due sets
+ *      too small to fill the GPU), their outputs going back to their token
+ *      rows.
  *
  * Conventions shared by every entry point
  *   - All pointers named *device* below are device pointers on the current
