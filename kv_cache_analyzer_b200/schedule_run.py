@@ -7,7 +7,8 @@ d = 128, BF16.  The analyzer scores token-sized blocks of the latent history,
 classify splits them 30/30/40, and the schedule covers T = 50 steps (5
 warm-up, Moderate every 2, Static every 4, 5 cool-down).  Each step scatters
 the fresh K/V of its due tokens into the carried cache and runs attention of
-their queries over the whole cache.  Reported, as one JSON line:
+their queries over the whole cache (split over key ranges where the
+library's choice for that due set says so).  Reported, as one JSON line:
 
 * the 50 steps' scatter + attention device time, against 50 full-attention
   steps (every token due) on the same shape, and the FLOP ratio;
