@@ -58,7 +58,8 @@ typedef enum {
     JANO_EALIGN = 3,        /* pointer not 16-byte aligned                    */
     JANO_EUNSUPPORTED = 4,  /* valid but not implemented (e.g. d not 64/128)  */
     JANO_ENONFINITE = 5,    /* device: a score was NaN or infinite            */
-    JANO_EINDEX = 6,        /* device: an index or level was out of range     */
+    JANO_EINDEX = 6,        /* device: an index or level out of range, or an
+                               index list not strictly ascending             */
     JANO_ETIMEOUT = 7,      /* device: a bounded internal wait gave up (a bug) */
     JANO_ECUDA = 8          /* a CUDA runtime call or launch failed           */
 } jano_status;
@@ -183,10 +184,11 @@ JANO_API jano_status jano_build_schedule(const uint8_t *block_levels, const jano
  * __device__ array of 1 MiB inside the library, which every GPU that loads
  * the library holds until the process exits.  It allocates nothing.
  *
- * Limit: the scratch the geometry needs (jano_build_schedule_workspace_bytes)
- * must not exceed 1 MiB, i.e. about 1.04 million tokens; larger geometries
- * return JANO_EUNSUPPORTED and launch nothing.  Other errors are those of
- * jano_build_schedule.
+ * Limit: the scratch the geometry needs (jano_build_schedule_workspace_bytes,
+ * align16(n_tokens) + 2 * align16(12 * ceil(n_tokens / 1024)) bytes) must not
+ * exceed 1 MiB, which holds geometries of at most 1,024,544 tokens; larger
+ * ones return JANO_EUNSUPPORTED before any CUDA call and launch nothing.
+ * Other errors are those of jano_build_schedule.
  * Set-up: the first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
  * before any stream capture.
@@ -208,10 +210,13 @@ JANO_API jano_status jano_build_schedule_noalloc(const uint8_t *block_levels, co
  * K/V of frozen tokens are kept and reused); zh 2.2 item 3; pt 2.B.
  *
  * k_act, v_act      device BF16 [n_act][heads][d].
- * idx               device int32 [n_act], distinct ids in [0, n_tokens)
- *                   (jano_build_schedule emits ascending ones).  An id out of
- *                   range raises JANO_EINDEX on the device error word and
- *                   its row is skipped.  Duplicate ids: unspecified winner.
+ * idx               device int32 [n_act], strictly ascending ids in
+ *                   [0, n_tokens) (what jano_build_schedule emits).  A row
+ *                   whose id is out of range or not above the previous
+ *                   row's id raises JANO_EINDEX on the device error word and
+ *                   is skipped, so an adjacent duplicate never races; after
+ *                   that error, which cache rows hold which values is
+ *                   unspecified if the list was not ascending.
  * k_cache, v_cache  device BF16 [n_tokens][heads][d]; must not overlap the
  *                   act buffers.  All four 16-byte aligned; heads*d % 8 == 0.
  * n_act == 0 is a no-op.
@@ -233,8 +238,11 @@ JANO_API jano_status jano_kv_scatter(const void *k_act, const void *v_act, const
  * q_act             device BF16 [n_act][heads][d] (the due tokens' queries,
  *                   in the order of idx).
  * k_cache, v_cache  device BF16 [n_tokens][heads][d].
- * idx               device int32 [n_act]: output row of each query; out of
- *                   range raises JANO_EINDEX and the row is skipped.
+ * idx               device int32 [n_act]: output row of each query,
+ *                   strictly ascending in [0, n_tokens) (what
+ *                   jano_build_schedule emits).  A row whose id is out of
+ *                   range or not above the previous row's id raises
+ *                   JANO_EINDEX and is not written.
  * out               device BF16 [n_tokens][heads][d]; only rows idx[] are
  *                   written.  May not alias the inputs.
  * d in {64, 128}; BF16 in, fp32 accumulate and softmax, BF16 out;
@@ -305,14 +313,15 @@ JANO_API int jano_active_attention_splits_on(int n_act, int n_tokens, int heads,
  * x        device BF16 [n_x][k] (e.g. the hidden states of all tokens).
  * gather   device int32 [m] or NULL; values in [0, n_x).  Without it m <= n_x.
  * w        device BF16 [n][k]: a linear layer's weight in [out][in] layout.
- * scatter  device int32 [m] or NULL; values in [0, n_out).  Without it
- *          m <= n_out.  Two active rows must not share a destination.
+ * scatter  device int32 [m] or NULL; strictly ascending values in
+ *          [0, n_out).  Without it m <= n_out.
  * out      device BF16 [n_out][n]; rows not written keep their contents.
  * k % 8 == 0 and n % 8 == 0 (JANO_EUNSUPPORTED otherwise); x, w, out
  * 16-byte aligned.  BF16 in, fp32 accumulation on the tensor cores, BF16
  * out (round to nearest even).  An index out of range raises JANO_EINDEX on
- * the device error word: a bad gather index reads a row of zeros, a bad
- * scatter index drops the row.  m == 0 is a no-op.
+ * the device error word: a bad gather index reads a row of zeros, a
+ * scatter index out of range or not above the previous one drops the row.
+ * m == 0 is a no-op.
  * ---------------------------------------------------------------------- */
 JANO_API jano_status jano_gather_gemm(const void *x, int n_x, const int32_t *gather, int m,
                                       const void *w, int n, int k, const int32_t *scatter,
@@ -332,7 +341,8 @@ JANO_API jano_status jano_gather_gemm(const void *x, int n_x, const int32_t *gat
  * jano_kv_scatter.  hd = heads * d.
  *
  * x        device BF16 [n_tokens][k], the hidden states of all tokens.
- * idx      device int32 [n_act], the active tokens (distinct, in [0, n_tokens)).
+ * idx      device int32 [n_act], the active tokens, strictly ascending in
+ *          [0, n_tokens) (a K/V row whose id breaks that is dropped).
  * w_qkv    device BF16 [3*hd][k]: the Q rows, then the K rows, then the V rows.
  * q_act    device BF16 [n_act][hd]; k_cache, v_cache device BF16 [n_tokens][hd].
  * hd must be a multiple of 128 and k of 8 (JANO_EUNSUPPORTED otherwise);

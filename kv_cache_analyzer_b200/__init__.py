@@ -174,7 +174,7 @@ def jano_build_schedule_noalloc(block_levels, geom, cfg, offsets, idx, idx_capac
                                 stream=None):
     """jano_build_schedule without a workspace argument: for callers that
     cannot allocate device memory.  The library's own 1 MiB device array
-    serves as scratch (geometries up to about 1.04 million tokens); calls
+    serves as scratch (geometries of at most 1,024,544 tokens); calls
     overlapping on the GPU race on it, and the first call on a device should
     come before any stream capture."""
     _check("jano_build_schedule_noalloc", lib().jano_build_schedule_noalloc(
@@ -374,17 +374,24 @@ def active_attention(q_act, k_cache, v_cache, idx, out, scale=None, stream=None,
 
 
 class SplitWorkspace:
-    """Device workspace of key-split attention for one stream, grown on demand."""
+    """Device workspaces of key-split attention, one per stream, each grown
+    on demand.  Launches on one stream are ordered, so reusing that stream's
+    buffer is safe; a launch on another stream gets a buffer of its own, so
+    concurrent split launches never share partials."""
 
     def __init__(self, device):
         self.device = torch.device(device)
-        self.buf = None
+        self.bufs = {}
 
     def get(self, nbytes: int, stream) -> torch.Tensor:
-        if self.buf is None or self.buf.numel() < nbytes:
-            with torch.cuda.stream(_torch_stream(stream)):
-                self.buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
-        return self.buf
+        ts = _torch_stream(stream)
+        key = int(ts.cuda_stream)
+        buf = self.bufs.get(key)
+        if buf is None or buf.numel() < nbytes:
+            with torch.cuda.stream(ts):
+                buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+            self.bufs[key] = buf
+        return buf
 
 
 def attention_auto(q_act, k_cache, v_cache, idx, n_act, n_tokens, heads, d, out, stream,

@@ -449,8 +449,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         const int qi = q0 + i * BM + row;
         int t_out = -1;
         if (qi < n_act) {
+            // idx contract: in range and strictly ascending; a row that breaks
+            // it is reported and not written
             t_out = __ldg(idx + qi);
-            if (t_out < 0 || t_out >= n_tokens) {
+            if (t_out < 0 || t_out >= n_tokens || (qi > 0 && __ldg(idx + qi - 1) >= t_out)) {
                 raise_error(err, JANO_EINDEX);
                 t_out = -1;
             }
@@ -471,7 +473,14 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (lane == 0) ptx::mbar_arrive(ctl.bar(L::bPFull + i));
         }
         // ------------------------------------------------------------ epilogue
-        if (ok && ctl.warp_wait(L::bOFull + i, 0)) {
+        const bool done = ok && ctl.warp_wait(L::bOFull + i, 0);
+        if constexpr (kSplit) {
+            // a CTA that gave up leaves a marker (l < 0, impossible for a sum of
+            // exponentials) instead of its partial, so the merge skips the row
+            if (!done && qi < n_act)
+                part_ml[((size_t)split * n_act + qi) * heads + head] = make_float2(-INFINITY, -1.0f);
+        }
+        if (done) {
             ptx::tc_fence_after();
             if constexpr (!kSplit) {
                 const float inv = 1.0f / l;
@@ -524,7 +533,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
 // Merge of the key-split partials: one warp per (query, head) row; lane
 // holds HD/32 consecutive columns.  With M = max_s m_s and w_s = 2^(m_s - M),
 //   out[idx[i], h] = sum_s w_s O_s / sum_s w_s l_s,
-// summed over the splits in order (deterministic).
+// summed over the splits in order (deterministic).  Rows with a missing
+// partial (a timed-out range) or a bad index are left untouched.
 template <int HD>
 __global__ void __launch_bounds__(256)
 attention_combine_kernel(const float* __restrict__ part_o, const float2* __restrict__ part_ml,
@@ -537,12 +547,20 @@ attention_combine_kernel(const float* __restrict__ part_o, const float2* __restr
     if (row >= rows) return;
     const int qi = (int)(row / heads), head = (int)(row % heads);
     const int t = __ldg(idx + qi);
-    if (t < 0 || t >= n_tokens) {
+    if (t < 0 || t >= n_tokens || (qi > 0 && __ldg(idx + qi - 1) >= t)) {
         if (lane == 0) raise_error(err, JANO_EINDEX);
         return;
     }
     float M = -INFINITY;
-    for (int z = 0; z < n_split; ++z) M = fmaxf(M, part_ml[z * rows + row].x);
+    bool missing = false;
+    for (int z = 0; z < n_split; ++z) {
+        const float2 ml = part_ml[z * rows + row];
+        missing |= ml.y < 0.0f;
+        M = fmaxf(M, ml.x);
+    }
+    // a key range whose CTA timed out (JANO_ETIMEOUT already raised) left no
+    // partial: the row is not written, as in the unsplit kernel
+    if (missing) return;
     float acc[E], L = 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;

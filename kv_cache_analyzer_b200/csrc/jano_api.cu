@@ -280,7 +280,7 @@ const char* jano_status_str(jano_status s) {
         case JANO_EALIGN: return "pointer not 16-byte aligned";
         case JANO_EUNSUPPORTED: return "unsupported configuration";
         case JANO_ENONFINITE: return "non-finite score";
-        case JANO_EINDEX: return "index or level out of range";
+        case JANO_EINDEX: return "index or level out of range, or indices not strictly ascending";
         case JANO_ETIMEOUT: return "device wait timed out";
         case JANO_ECUDA: return "CUDA error";
     }

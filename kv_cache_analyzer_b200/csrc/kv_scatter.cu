@@ -7,6 +7,11 @@
 // lanes move the row's 16-byte vectors with UNROLL independent K and V loads
 // in flight per lane before the stores.  Rows are grid-strided over a grid
 // sized to fill every SM.  No scratch memory.
+//
+// Index contract: idx strictly ascending (what the schedule emits).  A row
+// whose id is out of range, or not above the previous row's id (a duplicate
+// or a step back), raises JANO_EINDEX and is skipped, so an adjacent
+// duplicate never races; the extra load hits the line the warp just read.
 #include "jano_common.cuh"
 
 namespace jano {
@@ -25,7 +30,7 @@ kv_scatter_kernel(const uint4* __restrict__ k_act, const uint4* __restrict__ v_a
     const int nwarps = gridDim.x * kWarps;
     for (int i = warp; i < n_act; i += nwarps) {
         const int t = __ldg(idx + i);
-        if (t < 0 || t >= n_tokens) {
+        if (t < 0 || t >= n_tokens || (i > 0 && __ldg(idx + i - 1) >= t)) {
             if (lane == 0) raise_error(err, JANO_EINDEX);
             continue;
         }

@@ -315,7 +315,9 @@ projection_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
                 int dst_row = -1;
                 if (r < a.m) {
                     dst_row = sg.rowmap ? __ldg(sg.rowmap + r) : r;
-                    if (dst_row < 0 || dst_row >= sg.n_rows) {
+                    // scattered rows: in range and strictly ascending
+                    if (dst_row < 0 || dst_row >= sg.n_rows ||
+                        (sg.rowmap && r > 0 && __ldg(sg.rowmap + r - 1) >= dst_row)) {
                         raise_error(a.err, JANO_EINDEX);
                         dst_row = -1;
                     }

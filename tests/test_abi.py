@@ -177,3 +177,27 @@ def test_split_choice_on_a_given_sm_count(jl):
             for N in (128, 1024, 32760, 75600):
                 z = f(n, N, 4, 128, sms)
                 assert 1 <= z <= 16 and (z == 1 or ((N + 127) // 128) // z >= 8)
+
+
+def test_noalloc_limit_is_exactly_its_scratch(jl):
+    # The static scratch is 1 MiB: align16(n) + 2 * align16(12 * ceil(n / 1024))
+    # bytes for n tokens.  317 x 3232 = 1,024,544 tokens need exactly 1 MiB;
+    # one token more (a 1 x 1,024,545 row) needs 1,048,592 bytes.
+    L = jl.lib()
+    at = jl.Geometry(1, 317, 3232, (1, 1, 1), (1, 1, 1))
+    over = jl.Geometry(1, 1, 1_024_545, (1, 1, 1), (1, 1, 1))
+    assert at.n_tokens == 1_024_544 and over.n_tokens == 1_024_545
+    assert jl.jano_build_schedule_workspace_bytes(at.c()) == 1 << 20
+    assert jl.jano_build_schedule_workspace_bytes(over.c()) == (1 << 20) + 16
+    c = jl.Schedule(2, 1, 1, 1, 1).c()
+    nil = C.c_void_p(0)
+    g_over = over.c()
+    # one token over the limit: rejected before any CUDA call (no device needed)
+    assert L.jano_build_schedule_noalloc(nil, C.byref(g_over), C.byref(c), nil, nil, 10**9, nil,
+                                         nil) == 4
+    # at the limit the size check passes; the call then fails later for other
+    # reasons (no device here -> JANO_ECUDA, NULL buffers -> JANO_EINVAL), never
+    # with JANO_EUNSUPPORTED
+    g_at = at.c()
+    assert L.jano_build_schedule_noalloc(nil, C.byref(g_at), C.byref(c), nil, nil, 10**9, nil,
+                                         nil) in (1, 8)

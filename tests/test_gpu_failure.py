@@ -37,8 +37,12 @@ def inject_lib():
     P, i, f = C.c_void_p, C.c_int, C.c_float
     L.jano_active_attention.argtypes = [P, P, P, P, i, i, i, i, f, P, P]
     L.jano_qkv_project.argtypes = [P, i, P, i, P, i, i, P, P, P, P]
+    L.jano_active_attention_split.argtypes = [P, P, P, P, i, i, i, i, f, i, P, C.c_size_t, P, P]
+    L.jano_active_attention_workspace_bytes.argtypes = [i, i, i, i]
+    L.jano_active_attention_workspace_bytes.restype = C.c_size_t
     L.jano_get_device_error.argtypes = [P]
-    for fn in ("jano_active_attention", "jano_qkv_project", "jano_get_device_error"):
+    for fn in ("jano_active_attention", "jano_active_attention_split", "jano_qkv_project",
+               "jano_get_device_error"):
         getattr(L, fn).restype = C.c_int
     return L
 
@@ -76,6 +80,30 @@ def test_attention_wait_runs_out_and_reports_etimeout(inject_lib):
     assert code == ETIMEOUT, code
     assert wall < 30.0, wall
     assert L.jano_get_device_error(_stream()) == 0    # read and cleared
+
+
+def test_split_attention_timeout_leaves_rows_untouched(inject_lib):
+    # 384 keys = 3 key tiles in 2 ranges: range 0 takes tile 0 (two loads, none
+    # dropped) and completes; range 1 takes tiles 1-2, its third load is never
+    # issued and it times out.  The merge must then skip every row (one of its
+    # partials is missing) instead of reading the range's unwritten workspace,
+    # so `out` keeps its contents, as with the unsplit kernel.
+    L = inject_lib
+    gen = np.random.default_rng(2)
+    N, n_act, H, d, n_split = 384, 128, 1, 128, 2
+    q = synth.normal_bf16((n_act, H, d), 11).cuda()
+    kc = synth.normal_bf16((N, H, d), 12).cuda()
+    vc = synth.normal_bf16((N, H, d), 13).cuda()
+    ix = torch.from_numpy(np.sort(gen.choice(N, size=n_act, replace=False)).astype(np.int32)).cuda()
+    out = torch.full((N, H, d), 0.25, dtype=torch.bfloat16, device="cuda")
+    nb = L.jano_active_attention_workspace_bytes(n_act, H, d, n_split)
+    # garbage in the workspace, as a reused buffer would hold
+    ws = torch.full((nb // 4,), float("nan"), dtype=torch.float32, device="cuda")
+    assert L.jano_active_attention_split(_p(q), _p(kc), _p(vc), _p(ix), n_act, N, H, d, d ** -0.5,
+                                         n_split, _p(ws), nb, _p(out), _stream()) == 0
+    assert L.jano_get_device_error(_stream()) == ETIMEOUT
+    assert L.jano_get_device_error(_stream()) == 0
+    assert torch.all(out == 0.25)
 
 
 def test_projection_wait_runs_out_and_reports_etimeout(inject_lib):

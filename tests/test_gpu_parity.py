@@ -6,9 +6,13 @@ the KV-cache scatter.  Floating point: block scores within
 within max-abs 2e-2 and mean-rel 5e-3 (sum|gpu-ref| / sum|ref|) of the fp64
 values (BF16 in and out, fp32 accumulation and softmax).
 
-Every workload of the benchmark set runs at its full size; attention on the
-two video workloads is compared on sampled rows (first, last and seeded
-random ones) since the oracle computes one row in about a second there.
+Every workload of the benchmark set runs at its full size.  Attention on the
+two video workloads is compared on sampled rows, since the oracle takes up to
+a second per row there: at least 256 rows chosen so that every position of
+the kernel's grid is reached (both query tiles of a CTA's pair, all four
+32-row TMEM lane quarters, the first, last and evenly spaced CTAs, the
+ragged last pair), all heads of each row.  The oracle rows run concurrently
+on the host cores.
 """
 import math
 
@@ -18,7 +22,8 @@ import torch
 
 import oracle
 import synth
-from workloads import attention_case, attention_errors, latent, sample_rows, token_field, token_geometry
+from workloads import (attention_case, attention_errors, cta_position_rows, latent,
+                       oracle_attention_rows, sample_rows, token_field, token_geometry)
 
 pytestmark = pytest.mark.gpu
 
@@ -234,18 +239,45 @@ def _attention_check(J, q, kc, vc, idx, rows, scale=None):
     return mx, mr, out
 
 
+def attention_rows_for(name, n_act, seed):
+    """All rows for tiny; grid-position rows (>= 256) plus seeded random ones
+    for the others."""
+    if name == "tiny":
+        return np.arange(n_act, dtype=np.int32)
+    pos = cta_position_rows(n_act, n_ctas=32, seed=seed)
+    extra = sample_rows(n_act, 64, seed=seed + 1)
+    rows = np.unique(np.concatenate([pos, extra])).astype(np.int32)
+    assert rows.size >= min(256, n_act)
+    return rows
+
+
 @pytest.mark.parametrize("name", ALL)
 def test_attention_after_scatter_matches_oracle(J, name):
     c = attention_case(name)
     w, idx = c["w"], c["idx"]
     kc, vc = dev_bf16(c["k_stale"]), dev_bf16(c["v_stale"])
     J.kv_scatter(dev_bf16(c["k_act"]), dev_bf16(c["v_act"]), torch.from_numpy(idx).cuda(), kc, vc)
-    rows = sample_rows(idx.size, 10**9 if name in ("tiny", "image") else 6, seed=w.seed)
-    if name == "image":
-        rows = sample_rows(idx.size, 256, seed=w.seed)
-    mx, mr, _ = _attention_check(J, c["q_act"], kc.cpu(), vc.cpu(), idx, rows)
+    # the oracle's inputs come from the oracle's own scatter of the same rows
+    rk, rv = oracle.kv_scatter(synth.bits_of(c["k_act"]), synth.bits_of(c["v_act"]), idx,
+                               synth.bits_of(c["k_stale"]), synth.bits_of(c["v_stale"]))
+    rows = attention_rows_for(name, idx.size, w.seed)
+    N, H, d = kc.shape
+    out = torch.zeros(N, H, d, dtype=torch.bfloat16, device="cuda")
+    J.active_attention(dev_bf16(c["q_act"]), kc, vc, torch.from_numpy(idx).cuda(), out)
+    no_device_error(J)
+    ref = oracle_attention_rows(synth.bits_of(c["q_act"]), rk, rv, rows)
+    got = out.cpu()
+    g = got[torch.from_numpy(idx[rows]).long()].float().numpy()
+    mx, mr = attention_errors(g, ref)
     print(f"{name}: rows {rows.size}, max-abs {mx:.3e}, mean-rel {mr:.3e}")
     assert mx <= ATT_MAX_ABS and mr <= ATT_MEAN_REL
+    # per row as well: no single row may be far off while the mean hides it
+    per_row = np.abs(g - ref).reshape(rows.size, -1).max(axis=1)
+    assert per_row.max() <= ATT_MAX_ABS
+    # rows not in idx stay untouched (zero)
+    mask = torch.ones(N, dtype=torch.bool)
+    mask[torch.from_numpy(idx).long()] = False
+    assert torch.count_nonzero(got[mask].float()) == 0
 
 
 @pytest.mark.parametrize("N,n_act,H,d", [(1, 1, 1, 128), (127, 5, 2, 64), (129, 129, 1, 128),
@@ -342,3 +374,47 @@ def test_attention_deterministic_and_bad_index(J):
     assert J.device_error() == 6
     keep = np.delete(np.arange(n_act), 3)
     assert torch.equal(o[idx[keep]], outs[0][idx[keep]])
+
+
+# ---------------------------------------------------------------- idx contract
+# idx must be strictly ascending (what the schedule emits).  A row whose id is
+# not above the previous row's id (a duplicate or a step back) raises
+# JANO_EINDEX and is skipped; the other rows are computed as usual.
+BAD_IDX = np.array([0, 2, 2, 5, 4, 9, 11, 13], dtype=np.int32)   # rows 2 (dup) and 4 (back)
+BAD_ROWS = [2, 4]
+GOOD_ROWS = [0, 1, 3, 5, 6, 7]
+
+
+def test_kv_scatter_rejects_duplicate_and_descending_ids(J):
+    N, H, d = 16, 2, 64
+    kc = synth.normal_bf16((N, H, d), 41).cuda()
+    vc = synth.normal_bf16((N, H, d), 42).cuda()
+    before_k, before_v = kc.clone(), vc.clone()
+    ka = synth.normal_bf16((BAD_IDX.size, H, d), 43).cuda()
+    va = synth.normal_bf16((BAD_IDX.size, H, d), 44).cuda()
+    J.kv_scatter(ka, va, torch.from_numpy(BAD_IDX).cuda(), kc, vc)
+    assert J.device_error() == 6
+    good = BAD_IDX[GOOD_ROWS]
+    assert torch.equal(kc[good], ka[GOOD_ROWS]) and torch.equal(vc[good], va[GOOD_ROWS])
+    # token 2 holds row 1 (the duplicate row 2 was skipped); token 4 is untouched
+    rest = np.setdiff1d(np.arange(N), good)
+    assert torch.equal(kc[rest], before_k[rest]) and torch.equal(vc[rest], before_v[rest])
+
+
+@pytest.mark.parametrize("split", [1, 2])
+def test_attention_rejects_duplicate_and_descending_ids(J, split):
+    N, H, d = 300, 2, 128
+    q = synth.normal_bf16((BAD_IDX.size, H, d), 45)
+    k = synth.normal_bf16((N, H, d), 46)
+    v = synth.normal_bf16((N, H, d), 47)
+    out = torch.zeros(N, H, d, dtype=torch.bfloat16, device="cuda")
+    J.active_attention(dev_bf16(q), dev_bf16(k), dev_bf16(v), torch.from_numpy(BAD_IDX).cuda(), out,
+                       split=split)
+    assert J.device_error() == 6
+    ref = oracle.active_attention(synth.bits_of(q), synth.bits_of(k), synth.bits_of(v),
+                                  rows=np.array(GOOD_ROWS, dtype=np.int32))
+    got = out.cpu()[torch.from_numpy(BAD_IDX[GOOD_ROWS]).long()].float().numpy()
+    mx, mr = attention_errors(got, ref)
+    assert mx <= ATT_MAX_ABS and mr <= ATT_MEAN_REL
+    # token 4 (only named by the skipped row 4) stays unwritten
+    assert torch.count_nonzero(out[4].float()) == 0

@@ -19,6 +19,7 @@ import torch
 
 import oracle
 import synth
+from workloads import cta_position_rows, oracle_gemm_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -44,7 +45,7 @@ def f32(bits):
 
 def check_rows(got_bits, x_bits, w_bits, src_rows, label=""):
     """got_bits [r][n] BF16 bits of the GPU rows; src_rows the x rows they read."""
-    ref = oracle.gather_gemm(x_bits, w_bits, np.asarray(src_rows, dtype=np.int32))
+    ref = oracle_gemm_rows(x_bits, w_bits, np.asarray(src_rows, dtype=np.int32))
     absdot = np.abs(f32(x_bits)[src_rows]) @ np.abs(f32(w_bits)).T
     got = f32(got_bits)
     err = np.abs(got - ref)
@@ -145,7 +146,9 @@ def test_qkv_project_equals_gather_gemm_then_kv_scatter(J):
 
 def test_qkv_project_large_video_sampled_rows(J):
     # the large video workload's shapes: 75,600 tokens, hidden 5120 = 40 heads x 128,
-    # the 18,900 Active tokens; rows compared: first, last and seeded random ones
+    # the 18,900 Active tokens; rows compared (every output column of each):
+    # one in each 128-row half and 32-row TMEM lane quarter of 32 spread
+    # 256-row tiles, first, last (ragged last tile) and seeded random ones
     N, heads, d = 75600, 40, 128
     hd = k = heads * d
     gen = np.random.default_rng(4)
@@ -158,7 +161,9 @@ def test_qkv_project_large_video_sampled_rows(J):
     vc = torch.zeros((N, hd), dtype=torch.bfloat16, device="cuda")
     J.qkv_project(x.cuda(), torch.from_numpy(idx).cuda(), w.cuda(), q, kc, vc)
     no_device_error(J)
-    rows = np.unique(np.concatenate([[0, n_act - 1], gen.choice(n_act, size=4, replace=False)]))
+    rows = np.unique(np.concatenate([cta_position_rows(n_act, n_ctas=32, seed=5),
+                                     gen.choice(n_act, size=16, replace=False)]))
+    assert rows.size >= 256
     xb, wb = synth.bits_of(x), synth.bits_of(w)
     src = idx[rows]
     check_rows(synth.bits_of(q.cpu())[rows], xb, wb[:hd], src, "large q")
@@ -179,3 +184,23 @@ def test_bad_indices_raise_eindex(J):
     J.gather_gemm(x[:8].contiguous(), w, out2, scatter=s)
     assert J.device_error() == 6
     no_device_error(J)                                            # the error word was cleared
+
+
+def test_qkv_project_rejects_duplicate_and_descending_ids(J):
+    # K/V rows go to cache rows idx[i]: ids must be strictly ascending; rows 2
+    # (duplicate) and 4 (step back) raise JANO_EINDEX and write no K/V row
+    N, hd, k = 16, 128, 64
+    idx = np.array([0, 2, 2, 5, 4, 9, 11, 13], dtype=np.int32)
+    good = [0, 1, 3, 5, 6, 7]
+    x = synth.normal_bf16((N, k), seed=51)
+    w = synth.linear_weight_bf16(3 * hd, k, seed=52)
+    q = torch.zeros((idx.size, hd), dtype=torch.bfloat16, device="cuda")
+    kc0 = synth.normal_bf16((N, hd), seed=53)
+    kc, vc = kc0.clone().cuda(), kc0.clone().cuda()
+    J.qkv_project(x.cuda(), torch.from_numpy(idx).cuda(), w.cuda(), q, kc, vc)
+    assert J.device_error() == 6
+    xb, wb = synth.bits_of(x), synth.bits_of(w)
+    kb = synth.bits_of(kc.cpu())
+    check_rows(kb[idx[good]], xb, wb[hd:2 * hd], idx[good], "k of the valid rows")
+    # token 4 is named only by the skipped row: unchanged
+    np.testing.assert_array_equal(kb[4], synth.bits_of(kc0)[4])
