@@ -24,6 +24,19 @@ the schedule's larger due sets (Active + Moderate, and every token).
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead, on
 a bounded sample of the same workload, extrapolated stage by stage to the
 full workload.
+
+Other measurements, each printing its own JSON line (``--mode``):
+
+    --workload schedule50     the 50-step interleaved schedule with the KV cache
+                              carried across steps, against 50 full steps, and the
+                              active-fraction sweep on the same shape
+    --mode splits             attention TFLOP/s for every key-split count of a few
+                              due sets (the data the split choice was fitted to)
+    --mode sharded            per-rank work of the head-sharded step, one rank at a
+                              time on this GPU (W = --ranks)
+    --mode projection         the projections of the active rows alone
+    --mode spectral           the FFT baseline score beside the analyzer and a
+                              plain read, L2 cleaned before each launch
 """
 from __future__ import annotations
 
@@ -61,7 +74,16 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def workload_config(w):
+def n_active_of(w) -> int:
+    """Due tokens of the step the bench times (the first interleaved step:
+    the Active level, frac_active of the tokens in basis points, floored)."""
+    return int(round(w.frac_active * 10000)) * w.n_tokens // 10000
+
+
+def workload_config(w, world: int = 1):
+    """The `config` of the JSON line: the same dict for both arms."""
+    cache_gb = 2.0 * w.n_tokens * w.heads * w.d * 2 / 1e9
+    act_gb = 3.0 * n_active_of(w) * w.heads * w.d * 2 / 1e9
     return {
         "workload": f"{w.name}: latent {list(w.latent_shape)} fp32, blocks {list(w.block)}, "
                     f"{w.n_tokens} tokens x {w.heads} heads x d={w.d} BF16, "
@@ -71,7 +93,18 @@ def workload_config(w):
         "latent": list(w.latent_shape), "block": list(w.block), "patch": list(w.patch),
         "schedule": {"T": w.T, "warmup": w.warmup, "cooldown": w.cooldown,
                      "period_moderate": w.period_moderate, "period_static": w.period_static},
+        "n_active": n_active_of(w), "global_batch": world, "parallelism": f"replicas x{world}",
+        "l2": f"no flush: the per-step working set (K/V cache {cache_gb:.2f} GB, Q/K/V act "
+              f"{act_gb:.2f} GB) is larger than the 126 MB L2",
     }
+
+
+def host_cores() -> int:
+    """Host threads this process may run on."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
 
 
 # ------------------------------------------------------------------ ranks
@@ -181,45 +214,69 @@ def oracle_inputs(inp, k_cache, v_cache, n_act):
             "va": synth.bits_of(inp["v_act"])}
 
 
-def cpu_oracle_step_time(w, inp, bits, budget_rows=8, rng_seed=0):
-    """Time the oracle stage by stage on a bounded sample, extrapolate each
-    stage to the full workload; returns (seconds per full step, FLOPs, sample
-    text).  `bits` holds the BF16 bit arrays of oracle_inputs (the scatter
-    writes into its caches in place)."""
+def _oracle_attention_rows(bits, rows, threads):
+    """oracle.active_attention on `rows`, cut into chunks run by `threads`
+    host threads (each chunk is the unchanged single-threaded oracle; ctypes
+    releases the GIL around the C call)."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    if threads <= 1:
+        return oracle.active_attention(bits["qb"], bits["kb"], bits["vb"], rows=rows)
+    parts = np.array_split(rows, min(threads, rows.size))
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        outs = list(ex.map(lambda r: oracle.active_attention(bits["qb"], bits["kb"], bits["vb"], rows=r),
+                           parts))
+    return np.concatenate(outs, axis=0)
+
+
+def cpu_oracle_step_time(w, inp, bits, attn_rows, threads=1, rng_seed=0):
+    """Time the oracle stage by stage: block scores, classify, schedule and
+    the KV scatter over the full workload, attention on `attn_rows` sampled
+    active rows (all heads, all keys) spread over `threads` host threads,
+    extrapolated linearly to every active row.  Returns a dict with the
+    extrapolated seconds per full step, the step's FLOPs, the wall time of
+    the sampled step and a text describing the sample.  `bits` holds the BF16
+    bit arrays of oracle_inputs (the scatter writes into its caches)."""
     import oracle
     oracle.build()
     N, H, d = w.n_tokens, w.heads, w.d
     lat = inp["lat"].numpy()
     field = inp["field"].numpy()
-    est = 0.0
-    parts = []
-    # a1 on one frame-block slab of all snapshots/channels
-    bf = w.block[0]
-    slab = np.ascontiguousarray(lat[:, :, :bf])
-    t = time.perf_counter(); oracle.block_scores(slab, w.block); dt = time.perf_counter() - t
-    est += dt * (w.F / bf); parts.append(f"scores {bf}/{w.F} frames")
-    # a2 + a3 in full
+    t_all = time.perf_counter()
     t = time.perf_counter()
+    oracle.block_scores(lat, w.block)
     lv = oracle.classify(field, w.frac_active, w.frac_static)
     off, idx, _ = oracle.build_schedule(lv, (w.F, w.H, w.W), w.patch, w.patch, w.T, w.warmup,
                                         w.cooldown, w.period_moderate, w.period_static)
-    est += time.perf_counter() - t; parts.append("classify+schedule full")
     n_act = int(off[w.warmup + 1] - off[w.warmup])
     sel = idx[off[w.warmup]:off[w.warmup + 1]]
-    # a4 on 256 rows, in place
-    m = min(256, n_act)
-    t = time.perf_counter()
-    oracle.kv_scatter(bits["ka"][:m], bits["va"][:m], sel[:m], bits["kb"], bits["vb"], inplace=True)
-    dt = time.perf_counter() - t
-    est += dt * n_act / m; parts.append(f"scatter {m} rows")
-    # a5 on budget_rows rows x all heads x all keys
+    oracle.kv_scatter(bits["ka"][:n_act], bits["va"][:n_act], sel, bits["kb"], bits["vb"], inplace=True)
+    est = time.perf_counter() - t
     g = np.random.default_rng(rng_seed)
-    rows = np.sort(g.choice(n_act, size=min(budget_rows, n_act), replace=False)).astype(np.int32)
-    t = time.perf_counter(); oracle.active_attention(bits["qb"], bits["kb"], bits["vb"], rows=rows)
+    rows = np.sort(g.choice(n_act, size=min(attn_rows, n_act), replace=False)).astype(np.int32)
+    t = time.perf_counter()
+    _oracle_attention_rows(bits, rows, threads)
     dt = time.perf_counter() - t
-    est += dt * n_act / rows.size; parts.append(f"attention {rows.size} rows x {H} heads x {N} keys")
-    flops = 4.0 * n_act * N * d * H
-    return est, flops, "; ".join(parts) + " (single-threaded fp64 C, extrapolated per stage)"
+    est += dt * n_act / rows.size
+    return {"seconds": est, "flops": 4.0 * n_act * N * d * H, "wall_s": time.perf_counter() - t_all,
+            "sample": f"block scores, classify, schedule and scatter over the full workload; "
+                      f"attention on {rows.size} of {n_act} active rows x {H} heads x {N} keys, "
+                      f"extrapolated to every active row (fp64 C oracle, {threads} host "
+                      f"thread{'s' if threads > 1 else ''})"}
+
+
+def cpu_baseline(w, inp, bits, cores, rng_seed=0):
+    """The oracle on all host cores (attention rows over a thread pool) and
+    single-threaded, each on a bounded sample (tens of seconds at most)."""
+    multi = cpu_oracle_step_time(w, inp, bits, attn_rows=min(512, max(16, 4 * cores)), threads=cores,
+                                 rng_seed=rng_seed)
+    single = cpu_oracle_step_time(w, inp, bits, attn_rows=4, threads=1, rng_seed=rng_seed + 1)
+    return {"value": multi["flops"] / multi["seconds"] / 1e12, "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle", "sample": multi["sample"], "extrapolated": True,
+            "full_step_s_extrapolated": multi["seconds"], "wall_s": multi["wall_s"],
+            "single_thread": {"value": single["flops"] / single["seconds"] / 1e12, "unit": "TFLOP/s",
+                              "cores": 1, "sample": single["sample"], "extrapolated": True,
+                              "full_step_s_extrapolated": single["seconds"], "wall_s": single["wall_s"]}}
 
 
 def measure_projections(J, hp, step, stream, pk, reps=10, cpu_rows=0):
@@ -372,26 +429,32 @@ def run_reference(args, w, rank, world):
         return 0
     inp, k_cache, v_cache, n_cap = make_inputs(w)
     bits = oracle_inputs(inp, k_cache, v_cache, n_cap)
-    # attention rows per step: the bounded sample shrinks with the step count
-    # so that the whole run stays within a few minutes (about 2.3 s per row)
-    rows = args.ref_rows if args.ref_rows > 0 else max(1, min(8, 60 // max(1, args.steps + args.warmup)))
-    times = []
-    flops = None
-    sample = ""
+    cores = host_cores()
+    # attention rows per sampled step: sized so that the whole run stays
+    # within a few minutes (about 2 s of one core per row of the large step)
+    rows = args.ref_rows if args.ref_rows > 0 else \
+        max(1, min(512, (90 * cores) // (2 * max(1, args.steps + args.warmup))))
+    est, walls = [], []
+    res = None
     for i in range(args.warmup + args.steps):
-        t0 = time.perf_counter()
-        est, flops, sample = cpu_oracle_step_time(w, inp, bits, budget_rows=rows, rng_seed=i)
+        res = cpu_oracle_step_time(w, inp, bits, attn_rows=rows, threads=cores, rng_seed=i)
         if i >= args.warmup:
-            times.append(est)
-        log(f"reference step {i}: estimated full step {est:.1f} s (wall {time.perf_counter()-t0:.1f} s)")
-    t = statistics.mean(times)
-    value = flops / t / 1e12
+            est.append(res["seconds"])
+            walls.append(res["wall_s"])
+        log(f"reference step {i}: sampled step {res['wall_s']:.1f} s, "
+            f"extrapolated full step {res['seconds']:.1f} s")
+    t = statistics.mean(est)
+    value = res["flops"] / t / 1e12
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+            "steps": args.steps, "warmup": args.warmup,
+            # what was run and timed: one sampled step (the value comes from
+            # its per-stage extrapolation to the full step, given beside it)
+            "ms_per_step": statistics.mean(walls) * 1e3, "ms_per_step_kind": "sampled step (wall)",
+            "extrapolated": True, "full_step_ms_extrapolated": t * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(w), "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-                             "sample": sample},
+            "data": "synthetic", "config": workload_config(w, world), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": res["sample"], "extrapolated": True},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -515,11 +578,8 @@ def run_gpu(args, w, rank, world, local_rank, dist):
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        t0 = time.perf_counter()
         bits = oracle_inputs(inp, k_cache, v_cache, n_cap)
-        est, fl, sample = cpu_oracle_step_time(w, inp, bits, budget_rows=args.ref_rows if args.ref_rows > 0 else 8)
-        cpu = {"value": fl / est / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-               "sample": sample, "wall_s": time.perf_counter() - t0}
+        cpu = cpu_baseline(w, inp, bits, host_cores())
 
     next_rows = None
     if not args.no_next:
@@ -528,12 +588,8 @@ def run_gpu(args, w, rank, world, local_rank, dist):
         next_rows.update(measure_fft_score(J, hp, stream, pk))
         next_rows.update(measure_attention_sizes(J, hp, stream, pk))
 
-    cfg = workload_config(w)
-    cache_gb = 2.0 * w.n_tokens * w.heads * w.d * 2 / 1e9
-    act_gb = 3.0 * n_cap * w.heads * w.d * 2 / 1e9
-    cfg.update({"n_active": n_act, "global_batch": world, "parallelism": f"replicas x{world}",
-                "l2": f"no flush: the per-step working set (K/V cache {cache_gb:.2f} GB, Q/K/V act "
-                      f"{act_gb:.2f} GB) is larger than the 126 MB L2"})
+    cfg = workload_config(w, world)
+    assert cfg["n_active"] == n_act, (cfg["n_active"], n_act)
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -544,6 +600,304 @@ def run_gpu(args, w, rank, world, local_rank, dist):
                                           "bf16_tflops": pk["bf16_tflops"],
                                           "bf16_tflops_sustained": bf16_sus}}
     print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ other measurements
+def _events_ms(fn, stream, reps, warm=2, pick="median"):
+    """Device time of fn() on `stream` by CUDA events (after `warm` calls)."""
+    import torch
+    for _ in range(warm):
+        fn()
+    ms = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        stream.synchronize()
+        ms.append(a.elapsed_time(b))
+    return min(ms) if pick == "min" else sorted(ms)[len(ms) // 2]
+
+
+def _raise_device_error(J, stream, what):
+    code = J.device_error(stream)
+    if code:
+        raise RuntimeError(f"device error in {what}: {J.jano_status_str(code)}")
+
+
+def run_schedule50(args):
+    """The 50-step interleaved schedule of the 32,760-token x 12-head workload
+    (5 warm-up, Moderate every 2, Static every 4, 5 cool-down), each step the
+    KV scatter of its due tokens into the carried cache and their attention
+    over the whole cache, against 50 full steps; then the active-fraction
+    sweep (attention of the top fraction of the token field).  Fresh
+    activations of a step come from seeded device pools by the indexing rule
+    of synth.step_rows."""
+    import torch
+    import synth
+    import kv_cache_analyzer_b200 as J
+    w = synth.WORKLOADS["schedule50"]
+    N, H, d = w.n_tokens, w.heads, w.d
+    dev = torch.device("cuda")
+    st = torch.cuda.current_stream()
+    geom = J.Geometry(w.F, w.H, w.W, w.block, w.patch)
+    sched = J.Schedule(w.T, w.warmup, w.cooldown, w.period_moderate, w.period_static)
+    lat = torch.from_numpy(synth.latent_history(w.K, w.C, w.F, w.H, w.W, seed=w.seed)).to(dev)
+    levels = J.classify(J.block_scores(lat, geom), w.frac_active, w.frac_static)
+    off, idx, _ = J.build_schedule(levels, geom, sched)
+    off_h = off.cpu().tolist()                       # one read-back per generation
+    g = torch.Generator(device=dev).manual_seed(5000)
+    pool = [torch.randn(N, H, d, device=dev, generator=g).bfloat16() for _ in range(3)]
+    kc = torch.randn(N, H, d, device=dev, generator=g).bfloat16()
+    vc = torch.randn(N, H, d, device=dev, generator=g).bfloat16()
+    out = torch.zeros(N, H, d, dtype=torch.bfloat16, device=dev)
+    ws = J.SplitWorkspace(dev)
+
+    def attend(q, toks, n):
+        J.attention_auto(q, kc, vc, toks, n, N, H, d, out, st, ws)
+
+    def run(tok_lists):
+        evs = []
+        for s, toks in enumerate(tok_lists):
+            rows = (toks.long() + 7 * s) % N
+            q, k, v = pool[0][rows], pool[1][rows], pool[2][rows]
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            J.kv_scatter(k, v, toks, kc, vc)
+            attend(q, toks, toks.numel())
+            b.record(st)
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs)
+
+    sched_lists = [idx[off_h[s]:off_h[s + 1]] for s in range(w.T)]
+    all_toks = torch.arange(N, dtype=torch.int32, device=dev)
+    run(sched_lists)
+    sched_ms = min(run(sched_lists) for _ in range(args.reps))
+    run([all_toks] * w.T)
+    full_ms = min(run([all_toks] * w.T) for _ in range(args.reps))
+    due = np.diff(np.array(off_h))
+    sched_flops = 4.0 * float(due.sum()) * N * d * H
+    full_flops = 4.0 * w.T * N * N * d * H
+
+    TF, TH, TW = w.grid
+    fld = torch.from_numpy(synth.token_field(TF, TH, TW, seed=w.seed * 10 + 1, sigma=w.field_sigma)).to(dev)
+    tgeom = J.Geometry(w.F, w.H, w.W, w.patch, w.patch)
+    sweep = []
+    for f in [float(x) for x in args.fractions.split(",")]:
+        lv = J.classify(fld, f, 1.0 - f)
+        # periods longer than the schedule: the first interleaved step holds only Active tokens
+        o, ix, _ = J.build_schedule(lv, tgeom, J.Schedule(w.T, w.warmup, w.cooldown, 10 * w.T, 10 * w.T))
+        a0, a1 = o[w.warmup:w.warmup + 2].cpu().tolist()
+        toks, n_act = ix[a0:a1], a1 - a0
+        q = pool[0][:n_act]
+        ms = _events_ms(lambda: attend(q, toks, n_act), st, args.reps, pick="min")
+        sweep.append({"fraction": f, "n_active": n_act, "ms": ms,
+                      "key_split": J.jano_active_attention_splits(n_act, N, H, d),
+                      "TFLOP/s": 4.0 * n_act * N * d * H / (ms * 1e-3) / 1e12})
+    _raise_device_error(J, st, "the schedule50 run")
+    print(json.dumps({
+        "mode": "schedule50",
+        "workload": f"schedule50: {N} tokens x {H} heads x d={d} BF16, 30/30/40 levels, T=50",
+        "schedule_ms": sched_ms, "full_ms": full_ms, "speedup_vs_full": full_ms / sched_ms,
+        "flop_ratio_full_over_schedule": full_flops / sched_flops,
+        "schedule_tflops": sched_flops / (sched_ms * 1e-3) / 1e12,
+        "full_tflops": full_flops / (full_ms * 1e-3) / 1e12,
+        "due_token_steps": int(due.sum()), "sweep": sweep}), flush=True)
+    return 0
+
+
+SPLIT_CASES = [(32760, 12, n) for n in (1638, 3276, 8190, 16380, 24570, 32760)] + \
+              [(75600, 5, 18900), (75600, 40, 18900), (75600, 40, 41580)]
+
+
+def run_splits(args):
+    """Attention TFLOP/s for every key-split count of a few due sets (keys,
+    heads, due queries; d = 128; random BF16 cache and queries, due rows a
+    random sorted subset), with the library's own choice beside them."""
+    import torch
+    import kv_cache_analyzer_b200 as J
+    d = 128
+    dev = torch.device("cuda")
+    st = torch.cuda.current_stream()
+    cases = [tuple(c) for c in args.case] if args.case else SPLIT_CASES
+    for N, H, n in cases:
+        g = torch.Generator(device=dev).manual_seed(0)
+        kc = torch.randn((N, H, d), generator=g, device=dev).bfloat16()
+        vc = torch.randn((N, H, d), generator=g, device=dev).bfloat16()
+        q = torch.randn((n, H, d), generator=g, device=dev).bfloat16()
+        idx = torch.sort(torch.randperm(N, device=dev, generator=g)[:n]).values.int()
+        out = torch.empty((N, H, d), dtype=torch.bfloat16, device=dev)
+        line = {"mode": "splits", "keys": N, "heads": H, "n_act": n,
+                "chosen": J.jano_active_attention_splits(n, N, H, d), "TFLOP/s": {}}
+        for z in args.splits:
+            if z > (N + 127) // 128:
+                continue
+            ws = torch.empty(max(16, J.jano_active_attention_workspace_bytes(n, H, d, z)),
+                             dtype=torch.uint8, device=dev)
+            ms = _events_ms(lambda: J.active_attention(q, kc, vc, idx, out, split=z, workspace=ws),
+                            st, args.reps)
+            line["TFLOP/s"][z] = round(4.0 * n * N * d * H / (ms * 1e-3) / 1e12, 1)
+        _raise_device_error(J, st, "the split sweep")
+        print(json.dumps(line), flush=True)
+        del kc, vc, q, out
+    return 0
+
+
+def run_sharded(args):
+    """Per-rank work of the head-sharded step (frame slabs for the analyzer,
+    head ranges for scatter and attention), measured one rank at a time on
+    this GPU: each rank's block scores, then (after the ranks' scores are
+    joined by a copy standing in for the all-gather, not timed) classify,
+    schedule, scatter and attention.  Random device inputs of the large
+    workload's shapes (--frames/--height/--width/--heads shrink it).  One
+    JSON line per W: every rank's time, the slowest, and T_1 / (W T_W)."""
+    import torch
+    import kv_cache_analyzer_b200 as J
+    from kv_cache_analyzer_b200.sharding import ShardedHotPath
+    K, C, F, H, W = 5, 16, args.frames, args.height, args.width
+    heads, d = args.heads, 128
+    frac_active, frac_static = 0.25, 0.45
+    lg = J.Geometry(F, H, W, (1, 4, 4), (1, 2, 2))
+    tg = J.Geometry(F, H, W, (1, 2, 2), (1, 2, 2))
+    sched = J.Schedule(50, 5, 5, 2, 4)
+    step = sched.warmup
+    N = tg.n_tokens
+    n_cap = int(round(frac_active * 10000)) * N // 10000
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev).manual_seed(0)
+    lat = torch.randn((K + 1, C, F, H, W), generator=g, device=dev)
+    field = torch.rand(tg.n_blocks, generator=g, device=dev)
+    acts = {k: torch.randn((n_cap, heads, d), generator=g, device=dev).to(torch.bfloat16)
+            for k in ("q_act", "k_act", "v_act")}
+    kc = torch.randn((N, heads, d), generator=g, device=dev).to(torch.bfloat16)
+    vc = torch.randn((N, heads, d), generator=g, device=dev).to(torch.bfloat16)
+    stream = torch.cuda.Stream()
+    base = None
+    for world in args.ranks:
+        shards = []
+        for r in range(world):
+            sh = ShardedHotPath(rank=r, world=world, K=K, C=C, latent_geom=lg, token_geom=tg,
+                                heads=heads, d=d, frac_active=frac_active, frac_static=frac_static,
+                                sched=sched, stream=stream, all_gather=None)
+            sh.set_activations(n_cap)
+            sh.load_latent(lat)
+            with torch.cuda.stream(stream):
+                sh.field.copy_(field)
+                for k, v in acts.items():
+                    getattr(sh, k).copy_(sh.head_slice(v))
+                sh.k_cache.copy_(sh.head_slice(kc))
+                sh.v_cache.copy_(sh.head_slice(vc))
+            shards.append(sh)
+        for sh in shards:
+            sh.run_local_scores()
+        with torch.cuda.stream(stream):
+            full = torch.cat([sh.local_scores() for sh in shards])
+            for sh in shards:
+                sh.scores.copy_(full)
+        for sh in shards:
+            sh.run_after_gather()
+        stream.synchronize()
+        for sh in shards:
+            sh.host_offsets = sh.offsets.cpu().tolist()
+        n_act = shards[0].due(step)[1]
+        per_rank = []
+        for sh in shards:
+            t_scores = _events_ms(sh.run_local_scores, stream, args.reps)
+
+            def rest(sh=sh):
+                sh.run_after_gather()
+                sh.run_head_kernels(step)
+            t_rest = _events_ms(rest, stream, args.reps)
+            per_rank.append({"rank": sh.rank, "heads": sh.heads, "frames": sh.f_own,
+                             "key_split": sh.last_split, "ms": t_scores + t_rest, "scores_ms": t_scores})
+        _raise_device_error(J, stream, "the sharded ranks")
+        t_max = max(p["ms"] for p in per_rank)
+        if base is None and world == 1:
+            base = t_max
+        line = {"mode": "sharded", "ranks": world, "n_active": n_act, "max_rank_ms": t_max,
+                "per_rank": per_rank}
+        if base is not None:
+            line["t1_over_w_tw"] = base / (world * t_max)
+        print(json.dumps(line), flush=True)
+        del shards
+        torch.cuda.empty_cache()
+    return 0
+
+
+def run_projection(args):
+    """The projections of the active rows alone: random BF16 hidden states
+    x [N][D] (N(0, 1)), weights W_qkv [3D][D] and W_o [D][D] (N(0, 1/D)), M
+    distinct active tokens; the fused Q/K/V projection (K and V straight into
+    the token-ordered cache) and the output projection scattered back."""
+    import torch
+    import kv_cache_analyzer_b200 as J
+    N, D, M = args.tokens, args.hidden, args.active
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev).manual_seed(0)
+    x = torch.randn((N, D), generator=g, device=dev).to(torch.bfloat16)
+    w_qkv = (torch.randn((3 * D, D), generator=g, device=dev) * D ** -0.5).to(torch.bfloat16)
+    w_o = (torch.randn((D, D), generator=g, device=dev) * D ** -0.5).to(torch.bfloat16)
+    idx = torch.sort(torch.randperm(N, device=dev, generator=g)[:M]).values.to(torch.int32)
+    q = torch.empty((M, D), dtype=torch.bfloat16, device=dev)
+    kc = torch.zeros((N, D), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    o_act = torch.randn((M, D), generator=g, device=dev).to(torch.bfloat16)
+    y = torch.zeros((N, D), dtype=torch.bfloat16, device=dev)
+    st = torch.cuda.current_stream()
+    ops = {"qkv_project": (lambda: J.qkv_project(x, idx, w_qkv, q, kc, vc), 2.0 * M * 3 * D * D),
+           "out_proj_scatter": (lambda: J.gather_gemm(o_act, w_o, y, scatter=idx), 2.0 * M * D * D)}
+    res = {"mode": "projection", "shape": {"tokens": N, "hidden": D, "active": M}}
+    for name, (fn, flops) in ops.items():
+        ms = _events_ms(fn, st, args.reps, warm=3)
+        res[name] = {"ms": ms, "TFLOP/s": flops / (ms * 1e-3) / 1e12}
+    _raise_device_error(J, st, "the projections")
+    print(json.dumps(res), flush=True)
+    return 0
+
+
+def run_spectral(args):
+    """The FFT baseline score of the last snapshot, the analyzer's block
+    scores over all K+1 snapshots and a plain torch.sum over the analyzer's
+    bytes, each launch alone with the L2 cleaned (a 256 MB read) before it,
+    on a random fp32 latent history (default: the large video latent)."""
+    import torch
+    import kv_cache_analyzer_b200 as J
+    C, F, H, W, K = args.channels, args.frames, args.height, args.width, 5
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev).manual_seed(0)
+    lat = torch.randn((K + 1, C, F, H, W), generator=g, device=dev)
+    geom = J.Geometry(F, H, W, (1, 4, 4), (1, 1, 1))
+    out = torch.empty(geom.n_blocks, device=dev)
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    st = torch.cuda.current_stream()
+    gc = geom.c()
+    snap = lat[K]
+    ops = {"fft_score": (lambda: J.jano_fft_scores(snap, C, gc, 1, out, st),
+                         4.0 * (snap.numel() + out.numel())),
+           "block_scores": (lambda: J.jano_block_scores(lat, K, C, gc, 0.5, 0.5, out, st),
+                            4.0 * (lat.numel() + out.numel())),
+           "plain_read": (lambda: torch.sum(lat), 4.0 * lat.numel())}
+    res = {"mode": "spectral", "shape": {"channels": C, "frames": F, "height": H, "width": W,
+                                          "block": [1, 4, 4], "steps": K, "cutoff": 1,
+                                          "n_blocks": geom.n_blocks}}
+    for name, (fn, nbytes) in ops.items():
+        for _ in range(3):
+            fn()
+        ms = []
+        for _ in range(args.reps):
+            flush.sum()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            fn()
+            b.record(st)
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        m = sorted(ms)[args.reps // 2]
+        res[name] = {"ms": m, "GB/s": nbytes / (m * 1e-3) / 1e9, "algorithmic_bytes": nbytes}
+    _raise_device_error(J, st, "the spectral run")
+    print(json.dumps(res), flush=True)
     return 0
 
 
@@ -561,7 +915,35 @@ def main():
                          "sized from --steps/--warmup for --impl reference)")
     ap.add_argument("--no-next", action="store_true",
                     help="skip the projections measured beside the step")
+    ap.add_argument("--mode", default="step",
+                    choices=["step", "schedule50", "splits", "sharded", "projection", "spectral"],
+                    help="step: the hot path's step (the contract line); others: see the docstring "
+                         "(--workload schedule50 selects schedule50)")
+    ap.add_argument("--reps", type=int, default=5, help="repetitions of the other modes")
+    ap.add_argument("--fractions", default="0.1,0.25,0.5,0.75,1.0", help="schedule50: sweep points")
+    ap.add_argument("--splits", type=int, nargs="+", default=[1, 2, 3, 4, 5, 6, 7, 8, 10, 12])
+    ap.add_argument("--case", type=int, nargs=3, action="append", metavar=("N", "HEADS", "N_ACT"),
+                    help="splits: a due set (repeatable)")
+    ap.add_argument("--ranks", type=int, nargs="+", default=[1, 2, 4, 8], help="sharded: W values")
+    ap.add_argument("--frames", type=int, default=21)
+    ap.add_argument("--height", type=int, default=90)
+    ap.add_argument("--width", type=int, default=160)
+    ap.add_argument("--heads", type=int, default=40)
+    ap.add_argument("--channels", type=int, default=16, help="spectral: latent channels")
+    ap.add_argument("--tokens", type=int, default=75600, help="projection: tokens")
+    ap.add_argument("--hidden", type=int, default=5120, help="projection: hidden size")
+    ap.add_argument("--active", type=int, default=18900, help="projection: active rows")
     args = ap.parse_args()
+
+    if args.workload == "schedule50" and args.mode == "step":
+        args.mode = "schedule50"
+    if args.mode != "step":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "mode": args.mode,
+                              "unavailable": "the reference arm times the hot path's step only"}))
+            return 0
+        return {"schedule50": run_schedule50, "splits": run_splits, "sharded": run_sharded,
+                "projection": run_projection, "spectral": run_spectral}[args.mode](args)
 
     import synth
     w = synth.WORKLOADS[args.workload]

@@ -6,6 +6,9 @@ import subprocess
 import sys
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+import synth  # noqa: E402
 
 
 def test_reference_arm_prints_the_contract_line():
@@ -21,8 +24,20 @@ def test_reference_arm_prints_the_contract_line():
         assert k in d, k
     assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
-    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == bench.host_cores()
     assert d["config"]["workload"].startswith("tiny")
+    # the same config dict as the GPU arm's, and the timed sample is what ms_per_step reports
+    assert d["config"] == bench.workload_config(synth.WORKLOADS["tiny"], 1)
+    assert d["extrapolated"] is True and d["ms_per_step"] > 0 and d["full_step_ms_extrapolated"] > 0
+
+
+def test_config_is_identical_for_both_arms():
+    import synth
+    for name in ("tiny", "large"):
+        w = synth.WORKLOADS[name]
+        c = bench.workload_config(w, 1)
+        assert c["n_active"] == bench.n_active_of(w)
+    assert bench.workload_config(synth.WORKLOADS["large"], 1)["n_active"] == 18900
 
 
 import pytest
@@ -41,6 +56,7 @@ def test_native_arm_prints_the_contract_line():
               "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
         assert k in d, k
     assert d["value"] > 0 and d["gpu_launches"] == 7 * 3
+    assert d["config"] == bench.workload_config(synth.WORKLOADS["tiny"], 1)
     r = d["roofline"]
     assert r["bound"] == "tensor" and r["peak"] > 0 and abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-9
     assert r["traffic"] is None                  # the DRAM record belongs to the large workload

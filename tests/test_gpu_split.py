@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synth
-from workloads import attention_errors, sample_rows
+from workloads import attention_errors, cta_position_rows, oracle_attention_rows, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -145,4 +145,32 @@ def test_small_due_set_of_the_sweep_takes_a_split(J):
     ref = oracle.active_attention(synth.bits_of(q), synth.bits_of(k), synth.bits_of(v), rows=rows)
     got = out.cpu()[torch.from_numpy(idx[rows]).long()].float().numpy()
     mx, mr = attention_errors(got, ref)
+    assert mx <= ATT_MAX_ABS and mr <= ATT_MEAN_REL, (mx, mr)
+
+
+@pytest.mark.parametrize("frac", [0.25, 0.5, 0.75, 1.0])
+def test_sweep_points_match_oracle(J, frac):
+    # the other points of the active-fraction sweep on the 32,760-token,
+    # 12-head shape: the top `frac` of the smooth per-token field is due (the
+    # sweep's first interleaved step), attention over the whole cache with the
+    # library's split choice for that due set (the 50% point splits keys)
+    w = synth.WORKLOADS["schedule50"]
+    N, H, d = w.n_tokens, w.heads, w.d
+    TF, TH, TW = w.grid
+    field = synth.token_field(TF, TH, TW, seed=w.seed * 10 + 1, sigma=w.field_sigma)
+    lv = oracle.classify(field, frac, 1.0 - frac)
+    idx = np.flatnonzero(lv == 3).astype(np.int32)
+    n_act = idx.size
+    assert n_act == int(round(frac * 10000)) * N // 10000
+    q = synth.normal_bf16((n_act, H, d), 700 + int(frac * 100))
+    k = synth.normal_bf16((N, H, d), 801)
+    v = synth.normal_bf16((N, H, d), 802)
+    split = J.jano_active_attention_splits(n_act, N, H, d)
+    out = _run(J, q, k, v, idx, None)
+    assert J.device_error() == 0
+    rows = cta_position_rows(n_act, n_ctas=16, seed=int(frac * 100))
+    ref = oracle_attention_rows(synth.bits_of(q), synth.bits_of(k), synth.bits_of(v), rows)
+    got = out.cpu()[torch.from_numpy(idx[rows]).long()].float().numpy()
+    mx, mr = attention_errors(got, ref)
+    print(f"sweep {frac:.2f}: n_act {n_act}, split {split}, rows {rows.size}, max-abs {mx:.2e}, mean-rel {mr:.2e}")
     assert mx <= ATT_MAX_ABS and mr <= ATT_MEAN_REL, (mx, mr)

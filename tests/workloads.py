@@ -5,6 +5,8 @@ test hands it the oracle's so both sides see identical inputs)."""
 from __future__ import annotations
 
 import functools
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
@@ -64,3 +66,54 @@ def attention_errors(gpu: np.ndarray, ref: np.ndarray):
     """(max-abs, mean-rel = sum|gpu-ref| / sum|ref|) over all elements."""
     diff = np.abs(gpu.astype(np.float64) - ref)
     return float(diff.max()), float(diff.sum() / np.abs(ref).sum())
+
+
+# ------------------------------------------------------------------ oracle in parallel
+def _pool_workers() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def oracle_attention_rows(q_bits, k_bits, v_bits, rows, scale=None, chunk=4):
+    """oracle.active_attention for the given active rows, the rows cut into
+    chunks that run concurrently on the host cores (the oracle is a C call
+    made through ctypes, which releases the GIL; each call is the unchanged
+    single-threaded oracle on its own rows)."""
+    rows = np.ascontiguousarray(rows, dtype=np.int32)
+    parts = [rows[i:i + chunk] for i in range(0, rows.size, chunk)]
+    with ThreadPoolExecutor(max_workers=_pool_workers()) as ex:
+        outs = list(ex.map(lambda r: oracle.active_attention(q_bits, k_bits, v_bits, scale=scale,
+                                                             rows=r), parts))
+    return np.concatenate(outs, axis=0)
+
+
+def oracle_gemm_rows(x_bits, w_bits, src_rows, chunk=2):
+    """oracle.gather_gemm for the given source rows, chunks run concurrently
+    on the host cores (as oracle_attention_rows)."""
+    src_rows = np.ascontiguousarray(src_rows, dtype=np.int32)
+    parts = [src_rows[i:i + chunk] for i in range(0, src_rows.size, chunk)]
+    with ThreadPoolExecutor(max_workers=_pool_workers()) as ex:
+        outs = list(ex.map(lambda r: oracle.gather_gemm(x_bits, w_bits, r), parts))
+    return np.concatenate(outs, axis=0)
+
+
+def cta_position_rows(n_act: int, n_ctas: int = 32, seed: int = 0, tile: int = 128,
+                      pair: int = 2, lanes: int = 32) -> np.ndarray:
+    """Active rows that reach every position of the attention kernel's grid:
+    for a spread of CTAs (first, last and evenly spaced ones between), one
+    row in each (query tile of the CTA's pair, 32-row TMEM lane quarter),
+    at a seeded lane; rows past n_act (the ragged last pair) are replaced by
+    the last rows that exist.  Row 0 and row n_act - 1 are always included."""
+    g = np.random.default_rng(seed)
+    per_cta = tile * pair
+    total = -(-n_act // per_cta)
+    ctas = np.unique(np.linspace(0, total - 1, min(n_ctas, total)).round().astype(int))
+    rows = [0, n_act - 1]
+    for c in ctas:
+        for t in range(pair):
+            for q in range(tile // lanes):
+                r = c * per_cta + t * tile + q * lanes + int(g.integers(lanes))
+                rows.append(r if r < n_act else n_act - 1 - int(g.integers(min(lanes, n_act))))
+    return np.unique(np.array(rows, dtype=np.int32))
