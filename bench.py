@@ -383,14 +383,17 @@ def measure_fft_score(J, hp, stream, pk, reps=10, cutoff=1):
     the analyzer under the same conditions: each launch alone, L2 cleaned
     before it (a 256 MB read, which leaves no dirty lines to write back), on
     the last warm-up snapshot x_K.  The FFT score reads one snapshot; the
-    analyzer reads all K+1.  A plain torch.sum over the analyzer's bytes,
-    timed the same way, gives the rate a single pass of that size reaches."""
+    analyzer reads all K+1.  The one-pass read ceiling of the analyzer's bytes
+    (jano_stream_sum, a kernel that only streams them) and a plain torch.sum,
+    timed the same way, give the rate a single pass of that size reaches."""
     import torch
     K, C = hp.K, hp.C
     x = hp.lat[K]
     out = torch.empty_like(hp.scores)
     geom = hp.lg.c()
     flush = torch.ones(64 << 20, dtype=torch.float32, device=hp.dev)
+    sms = torch.cuda.get_device_properties(hp.dev).multi_processor_count
+    partial = torch.empty(sms, dtype=torch.float32, device=hp.dev)
     snap_bytes = float(x.numel()) * 4 + out.numel() * 4
     lat_bytes = float(hp.lat.numel()) * 4 + out.numel() * 4
     ops = {
@@ -398,6 +401,8 @@ def measure_fft_score(J, hp, stream, pk, reps=10, cutoff=1):
         "block_scores_same_conditions": (lambda: J.jano_block_scores(hp.lat, K, C, geom, hp.w_t, hp.w_s,
                                                                      out, stream), lat_bytes),
         "plain_read_same_bytes": (lambda: torch.sum(hp.lat), float(hp.lat.numel()) * 4),
+        "stream_read_same_bytes": (lambda: J.jano_stream_sum(hp.lat, hp.lat.numel(), partial, sms, stream),
+                                   float(hp.lat.numel()) * 4),
     }
     res = {}
     for name, (fn, nbytes) in ops.items():
@@ -418,6 +423,10 @@ def measure_fft_score(J, hp, stream, pk, reps=10, cutoff=1):
         gbs = nbytes / (m * 1e-3) / 1e9
         res[name] = {"ms": m, "GB/s": gbs, "frac_of_hbm": gbs / pk["hbm_gbs"], "algorithmic_bytes": nbytes}
     res["fft_score"]["cutoff"] = cutoff
+    # the analyzer against the one-pass read ceiling of the same bytes (a kernel
+    # that only streams them: jano_stream_sum), both timed the same way
+    res["block_scores_same_conditions"]["frac_of_stream_read"] = (
+        res["stream_read_same_bytes"]["ms"] / res["block_scores_same_conditions"]["ms"])
     code = J.device_error(stream)
     if code:
         raise RuntimeError(f"device error in the FFT score: {J.jano_status_str(code)}")
@@ -586,6 +595,10 @@ def run_gpu(args, w, rank, world, local_rank, dist):
         next_rows = measure_projections(J, hp, step, stream, pk,
                                         cpu_rows=0 if args.no_cpu_baseline or world > 1 else 2)
         next_rows.update(measure_fft_score(J, hp, stream, pk))
+        # the analyzer's one-pass ceiling beside its in-step figure
+        kernels["block_scores"]["stream_read_ceiling_GB/s"] = next_rows["stream_read_same_bytes"]["GB/s"]
+        kernels["block_scores"]["frac_of_stream_read_alone"] = \
+            next_rows["block_scores_same_conditions"]["frac_of_stream_read"]
         next_rows.update(measure_attention_sizes(J, hp, stream, pk))
 
     cfg = workload_config(w, world)

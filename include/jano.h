@@ -138,7 +138,8 @@ JANO_API jano_status jano_block_scores_literal(const float *lat, int K, int C, c
  * scores  device fp32 [n_blocks] (any finite values).
  * levels  device uint8 [n_blocks], written with 1, 2 or 3.
  * A NaN or infinite score raises JANO_ENONFINITE on the device error word
- * and leaves `levels` unspecified.  One thread block; no scratch memory.
+ * and leaves `levels` unspecified.  One cluster of 8 thread blocks; no
+ * scratch memory.
  * ---------------------------------------------------------------------- */
 JANO_API jano_status jano_classify(const float *scores, int n_blocks, float frac_active,
                           float frac_static, uint8_t *levels, void *stream);
@@ -185,8 +186,8 @@ JANO_API jano_status jano_build_schedule(const uint8_t *block_levels, const jano
  * the library holds until the process exits.  It allocates nothing.
  *
  * Limit: the scratch the geometry needs (jano_build_schedule_workspace_bytes,
- * align16(n_tokens) + 2 * align16(12 * ceil(n_tokens / 1024)) bytes) must not
- * exceed 1 MiB, which holds geometries of at most 1,024,544 tokens; larger
+ * align16(n_tokens) + align16(12 * ceil(n_tokens / 1024)) bytes) must not
+ * exceed 1 MiB, which holds geometries of at most 1,036,416 tokens; larger
  * ones return JANO_EUNSUPPORTED before any CUDA call and launch nothing.
  * Other errors are those of jano_build_schedule.
  * Set-up: the first call on a device looks up the array's device address
@@ -399,6 +400,28 @@ JANO_API jano_status jano_random_scores(int n_blocks, uint64_t seed, float *scor
  * ---------------------------------------------------------------------- */
 JANO_API jano_status jano_fft_scores(const float *x, int C, const jano_geom *g, int cutoff,
                                      float *scores, void *stream);
+
+/* ------------------------------------------------------------------------
+ * jano_stream_sum -- one streaming pass over a float buffer: the read rate
+ * that the analyzer's single pass over its latent history is compared with.
+ * A calibration of the device, not a step of the method: the Jano pages have
+ * no counterpart.  The kernel does the least work a full read can do (a
+ * deep ring of 1-D bulk copies per CTA, the consumer threads adding the
+ * floats), so its time is the launch, the ramp-up of the memory pipeline,
+ * the stream itself and the tail, as for any one-pass kernel of that size.
+ *
+ * x          device fp32 [n], 16-byte aligned; n % 4 == 0 (n == 0 allowed).
+ * partial    device fp32 [n_partial], 16-byte aligned: partial[i] is the sum
+ *            (fp32, fixed order, deterministic) of the i-th contiguous share
+ *            of x, shares of ceil(n / 4 / n_partial) float4s (the last ones
+ *            may be shorter or empty, summing to 0).
+ * n_partial  CTAs, 1..65535; the SM count gives one CTA per SM.
+ * Errors: JANO_EINVAL (n < 0, n % 4, n_partial out of range, NULL),
+ * JANO_EALIGN, JANO_ECUDA; a timed-out internal wait raises JANO_ETIMEOUT on
+ * the device error word.
+ * ---------------------------------------------------------------------- */
+JANO_API jano_status jano_stream_sum(const float *x, long long n, float *partial, int n_partial,
+                                     void *stream);
 
 /* Synchronises `stream`, returns the first device-side error recorded on the
  * current device since the last call (JANO_OK if none) and clears it. */

@@ -41,7 +41,7 @@ EXPORTS = ("jano_block_scores", "jano_block_scores_literal", "jano_classify", "j
            "jano_build_schedule", "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention",
            "jano_active_attention_split", "jano_active_attention_workspace_bytes", "jano_active_attention_splits",
            "jano_active_attention_splits_on", "jano_gather_gemm", "jano_qkv_project", "jano_random_scores", "jano_fft_scores",
-           "jano_get_device_error", "jano_status_str", "jano_version")
+           "jano_stream_sum", "jano_get_device_error", "jano_status_str", "jano_version")
 
 
 class JanoError(RuntimeError):
@@ -91,6 +91,7 @@ def lib() -> C.CDLL:
         L.jano_qkv_project.argtypes = [P, i, P, i, P, i, i, P, P, P, P]
         L.jano_random_scores.argtypes = [i, C.c_uint64, P, P]
         L.jano_fft_scores.argtypes = [P, i, G, i, P, P]
+        L.jano_stream_sum.argtypes = [P, C.c_longlong, P, i, P]
         L.jano_get_device_error.argtypes = [P]
         L.jano_status_str.argtypes = [i]
         L.jano_status_str.restype = C.c_char_p
@@ -99,7 +100,7 @@ def lib() -> C.CDLL:
                    "jano_build_schedule_noalloc", "jano_kv_scatter", "jano_active_attention",
                    "jano_active_attention_split", "jano_get_device_error",
                    "jano_gather_gemm", "jano_qkv_project", "jano_random_scores", "jano_fft_scores",
-                   "jano_version"):
+                   "jano_stream_sum", "jano_version"):
             getattr(L, fn).restype = C.c_int
         _lib = L
     return _lib
@@ -174,7 +175,7 @@ def jano_build_schedule_noalloc(block_levels, geom, cfg, offsets, idx, idx_capac
                                 stream=None):
     """jano_build_schedule without a workspace argument: for callers that
     cannot allocate device memory.  The library's own 1 MiB device array
-    serves as scratch (geometries of at most 1,024,544 tokens); calls
+    serves as scratch (geometries of at most 1,036,416 tokens); calls
     overlapping on the GPU race on it, and the first call on a device should
     come before any stream capture."""
     _check("jano_build_schedule_noalloc", lib().jano_build_schedule_noalloc(
@@ -244,6 +245,23 @@ def jano_fft_scores(x, C_, geom, cutoff, scores, stream=None):
     _check("jano_fft_scores", lib().jano_fft_scores(
         _dev(x, "x", torch.float32), C_, geom, cutoff, _dev(scores, "scores", torch.float32),
         _stream(stream)))
+
+
+def jano_stream_sum(x, n, partial, n_partial, stream=None):
+    _check("jano_stream_sum", lib().jano_stream_sum(
+        _dev(x, "x", torch.float32), n, _dev(partial, "partial", torch.float32), n_partial,
+        _stream(stream)))
+
+
+def stream_sum(x: torch.Tensor, n_partial: int | None = None, out=None, stream=None) -> torch.Tensor:
+    """Partial sums of one streaming pass over the fp32 tensor x (the read-rate
+    calibration the analyzer is compared with); one CTA per SM by default."""
+    if n_partial is None:
+        n_partial = torch.cuda.get_device_properties(x.device).multi_processor_count
+    if out is None:
+        out = torch.empty(n_partial, dtype=torch.float32, device=x.device)
+    jano_stream_sum(x, x.numel(), out, n_partial, stream)
+    return out
 
 
 def jano_get_device_error(stream=None) -> int:

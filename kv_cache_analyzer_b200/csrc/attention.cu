@@ -205,7 +205,13 @@ __device__ __forceinline__ float exp64(const uint32_t (&s)[64], int valid, float
         if (kMask && e >= valid) a = 0.f;
         if (kMask && e + 1 >= valid) b = 0.f;
         acc[(e >> 1) & 3] = ptx::fadd2(acc[(e >> 1) & 3], ptx::f2(a, b));
+#ifdef JANO_PACK_INT
+        // BF16 by integer rounding (half up; p >= 0 and finite), packed with
+        // one byte permute: keeps the conversion on the integer pipes
+        pk[e >> 1] = __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
+#else
         pk[e >> 1] = ptx::pack_bf16(a, b);
+#endif
     }
     const uint64_t t = ptx::fadd2(ptx::fadd2(acc[0], acc[1]), ptx::fadd2(acc[2], acc[3]));
     float lo, hi;

@@ -11,10 +11,13 @@
 //
 // One thread-block cluster of 8 CTAs does the work with no global scratch:
 // each CTA histograms its eighth of the scores in shared memory (warp-
-// aggregated atomics, since most keys share their top digits), the 8
+// aggregated atomics, since most keys share their top digits; the first pass,
+// which has no prefix yet, builds one histogram for both targets), the 8
 // histograms are summed through distributed shared memory after a cluster
-// barrier, and every CTA picks the same digit.  Histograms are double
-// buffered so one cluster barrier per pass suffices.  The tie pass counts
+// barrier (each thread issues all its remote loads before using any), and
+// every CTA finds the same digit by a block-wide scan of the totals (two
+// bins per thread).  Histograms are double buffered so one cluster barrier
+// per pass suffices.  The tie pass counts
 // threshold ties per thread over a contiguous range, scans them inside the
 // CTA and across the 8 CTAs (again through distributed shared memory), then
 // writes the levels.  Each CTA keeps its slice of keys in shared memory
@@ -108,52 +111,93 @@ classify_kernel(const uint32_t* __restrict__ bits, int n, long long k_static,
         const int buf = pass & 1, shift = digit_shift(pass);
         const unsigned dmask = (1u << digit_width(pass)) - 1u;
         const uint32_t hmask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + digit_width(pass)));
-        for (int b = tid; b < 2 * kBins; b += kThreads) (&sh.hist[buf][0][0])[b] = 0u;
-        __syncthreads();
+        // pass 0 has no prefix yet: one histogram serves both targets
+        const bool one = pass == 0;
+        const int nh = one ? 1 : 2;
+        for (int b = tid; b < nh * kBins; b += kThreads) (&sh.hist[buf][0][0])[b] = 0u;
         const uint32_t p0 = sh.val[0] & hmask, p1 = sh.val[1] & hmask;
+        const unsigned need0 = sh.need[0], need1 = sh.need[1];
+        __syncthreads();
         for (int base = lo; base < hi; base += kThreads) {
             const int i = base + tid;
             const bool ok = i < hi;
             const uint32_t u = ok ? key(i) : 0u;
             const unsigned dg = (u >> shift) & dmask;
-            const bool m0 = ok && live0 && (u & hmask) == p0;
-            const bool m1 = ok && live1 && (u & hmask) == p1;
-            const unsigned a0 = __ballot_sync(0xFFFFFFFFu, m0);
-            const unsigned a1 = __ballot_sync(0xFFFFFFFFu, m1);
-            warp_agg_add(sh.hist[buf][0], a0, dg, m0);
-            warp_agg_add(sh.hist[buf][1], a1, dg, m1);
+            if (one) {
+                const bool m = ok && (live0 || live1);
+                warp_agg_add(sh.hist[buf][0], __ballot_sync(0xFFFFFFFFu, m), dg, m);
+            } else {
+                const bool m0 = ok && live0 && (u & hmask) == p0;
+                const bool m1 = ok && live1 && (u & hmask) == p1;
+                const unsigned a0 = __ballot_sync(0xFFFFFFFFu, m0);
+                const unsigned a1 = __ballot_sync(0xFFFFFFFFu, m1);
+                warp_agg_add(sh.hist[buf][0], a0, dg, m0);
+                warp_agg_add(sh.hist[buf][1], a1, dg, m1);
+            }
         }
         cluster.sync();            // all 8 local histograms of this pass are complete
-        for (int b = tid; b < 2 * kBins; b += kThreads) {
-            unsigned s = 0;
-            for (int r = 0; r < kCluster; ++r)
-                s += cluster.map_shared_rank(&sh.hist[buf][0][0], r)[b];
-            (&sh.hist[buf ^ 1][0][0])[b] = s;
+        // cluster-wide totals: every remote load of this thread issued before any is used
+        {
+            const unsigned* rem[kCluster];
+#pragma unroll
+            for (int r = 0; r < kCluster; ++r) rem[r] = cluster.map_shared_rank(&sh.hist[buf][0][0], r);
+            unsigned v[4][kCluster];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (k < 2 * nh) {
+#pragma unroll
+                    for (int r = 0; r < kCluster; ++r) v[k][r] = rem[r][tid + k * kThreads];
+                }
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (k < 2 * nh) {
+                    unsigned t = 0;
+#pragma unroll
+                    for (int r = 0; r < kCluster; ++r) t += v[k][r];
+                    (&sh.hist[buf ^ 1][0][0])[tid + k * kThreads] = t;
+                }
         }
         __syncthreads();
-        if (warp < 2 && (warp == 0 ? live0 : live1)) {
-            // lane owns 64 consecutive bins
-            const unsigned* t = sh.hist[buf ^ 1][warp] + 64 * lane;
-            unsigned s = 0;
-            for (int j = 0; j < 64; ++j) s += t[j];
-            unsigned incl = s;
+        // block-wide scan of the totals, two bins per thread, both targets at once
+        const unsigned* h0 = sh.hist[buf ^ 1][0];
+        const unsigned* h1 = sh.hist[buf ^ 1][one ? 0 : 1];
+        const unsigned a0 = h0[2 * tid], b0 = h0[2 * tid + 1];
+        const unsigned a1 = h1[2 * tid], b1 = h1[2 * tid + 1];
+        unsigned x0 = a0 + b0, x1 = a1 + b1;
+        unsigned i0 = x0, i1 = x1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y0 = __shfl_up_sync(0xFFFFFFFFu, i0, o);
+            const unsigned y1 = __shfl_up_sync(0xFFFFFFFFu, i1, o);
+            if (lane >= o) { i0 += y0; i1 += y1; }
+        }
+        if (lane == 31) { sh.wsum[0][warp] = i0; sh.wsum[1][warp] = i1; }
+        __syncthreads();
+        if (warp == 0) {
+            const unsigned w0 = sh.wsum[0][lane], w1 = sh.wsum[1][lane];
+            unsigned j0 = w0, j1 = w1;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const unsigned y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-                if (lane >= o) incl += y;
+                const unsigned y0 = __shfl_up_sync(0xFFFFFFFFu, j0, o);
+                const unsigned y1 = __shfl_up_sync(0xFFFFFFFFu, j1, o);
+                if (lane >= o) { j0 += y0; j1 += y1; }
             }
-            const unsigned need = sh.need[warp];
-            const unsigned excl = incl - s;
-            if (excl <= need && need < incl) {
-                unsigned acc = excl;
-                int dg = 64 * lane;
-                for (int j = 0; j < 64; ++j) {
-                    if (acc + t[j] > need) { dg = 64 * lane + j; break; }
-                    acc += t[j];
-                }
-                sh.val[warp] |= (uint32_t)dg << shift;
-                sh.need[warp] = need - acc;
-            }
+            __syncwarp();
+            sh.wsum[0][lane] = j0 - w0;       // exclusive prefix of the warp totals
+            sh.wsum[1][lane] = j1 - w1;
+        }
+        __syncthreads();
+        // the one thread whose two bins hold rank `need` fixes the digit
+        const unsigned e0 = sh.wsum[0][warp] + i0 - x0, e1 = sh.wsum[1][warp] + i1 - x1;
+        if (live0 && e0 <= need0 && need0 < e0 + x0) {
+            const bool first = need0 < e0 + a0;
+            sh.val[0] |= (uint32_t)(2 * tid + (first ? 0 : 1)) << shift;
+            sh.need[0] = need0 - e0 - (first ? 0u : a0);
+        }
+        if (live1 && e1 <= need1 && need1 < e1 + x1) {
+            const bool first = need1 < e1 + a1;
+            sh.val[1] |= (uint32_t)(2 * tid + (first ? 0 : 1)) << shift;
+            sh.need[1] = need1 - e1 - (first ? 0u : a1);
         }
         __syncthreads();
     }

@@ -257,6 +257,15 @@ jano_status jano_fft_scores(const float* x, int C, const jano_geom* g, int cutof
     return from_cuda(launch_fft_scores(x, C, *g, cutoff, scores, static_cast<cudaStream_t>(stream)));
 }
 
+jano_status jano_stream_sum(const float* x, long long n, float* partial, int n_partial, void* stream) {
+    if (n < 0 || n % 4 || n_partial < 1 || n_partial > 65535 || !partial) return JANO_EINVAL;
+    if (n > 0 && !x) return JANO_EINVAL;
+    if (!aligned16(x) || !aligned16(partial)) return JANO_EALIGN;
+    int* err = device_error_word();
+    if (!err) return JANO_ECUDA;
+    return from_cuda(launch_stream_sum(x, n, partial, n_partial, err, static_cast<cudaStream_t>(stream)));
+}
+
 jano_status jano_get_device_error(void* stream) {
     int* err = device_error_word();
     if (!err) return JANO_ECUDA;

@@ -88,6 +88,8 @@ cudaError_t launch_projection(const void* x, int n_x, const int32_t* gather, int
                               cudaStream_t st);
 int projection_tile_n(int n, int seg_w, int n_seg);
 cudaError_t launch_random_scores(int n, uint64_t seed, float* scores, cudaStream_t st);
+cudaError_t launch_stream_sum(const float* x, long long n, float* partial, int n_partial, int* err,
+                              cudaStream_t st);
 
 namespace ptx {
 

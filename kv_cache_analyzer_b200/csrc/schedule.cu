@@ -10,13 +10,14 @@
 // so no step has to wait on another and no tile on another:
 //   1. count   one CTA per 1024-token tile: token level (from the block map)
 //              stored to scratch, per-level counts of the tile via warp ballots;
-//   2. scan    one CTA: per-level exclusive prefixes over tiles, per-step
-//              totals and the offsets[] prefix over steps;
-//   3. write   one CTA per (tile, 8 steps): the tile's tokens ranked once in
-//              each of the four possible due sets (ballot + popc + one warp
-//              scan per set), then ascending stores of the due ids per step.
-// Scratch (caller-provided): token levels [n_tokens] u8, counts/prefixes
-// [3][n_tiles] int32 each.
+//   2. write   one CTA per tile: its per-level prefix over the earlier tiles
+//              and the level totals by a block reduction over the tile counts,
+//              the step offsets in closed form from those totals, the tile's
+//              tokens ranked once in each of the four possible due sets
+//              (ballot + popc + one warp scan per set), then ascending stores
+//              of the due ids of every step.
+// Scratch (caller-provided): token levels [n_tokens] u8 and tile counts
+// [3][n_tiles] int32, each part 16-byte aligned.
 #include "jano_common.cuh"
 
 namespace jano {
@@ -35,7 +36,6 @@ struct Geo {
 struct Ws {
     uint8_t* tok;                 // [n_tokens]
     int* cnt;                     // [3][n_tiles]   (level-1 index)
-    int* pre;                     // [3][n_tiles]
 };
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
@@ -46,8 +46,6 @@ Ws carve(void* base, long long n_tokens, int n_tiles) {
     w.tok = reinterpret_cast<uint8_t*>(p);
     p += align16((size_t)n_tokens);
     w.cnt = reinterpret_cast<int*>(p);
-    p += align16(sizeof(int) * 3 * (size_t)n_tiles);
-    w.pre = reinterpret_cast<int*>(p);
     return w;
 }
 
@@ -97,64 +95,65 @@ count_kernel(const uint8_t* __restrict__ block_levels, Geo g, int n_tokens,
     }
 }
 
-__global__ void __launch_bounds__(kTile)
-scan_kernel(Ws ws, int n_tiles, jano_sched_cfg c, int32_t* __restrict__ offsets) {
-    __shared__ int wsum[32];
-    __shared__ int s_tot[3];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // per level: exclusive prefix of the tile counts, chunk by chunk
-    for (int l = 0; l < 3; ++l) {
-        int run = 0;
-        for (int base = 0; base < n_tiles; base += kTile) {
-            const int i = base + tid;
-            const int v = i < n_tiles ? ws.cnt[l * n_tiles + i] : 0;
-            int incl = v;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            if (lane == 31) wsum[warp] = incl;
-            __syncthreads();
-            int wpre = 0, tot = 0;
-            for (int w = 0; w < 32; ++w) {
-                if (w < warp) wpre += wsum[w];
-                tot += wsum[w];
-            }
-            if (i < n_tiles) ws.pre[l * n_tiles + i] = run + wpre + incl - v;
-            run += tot;
-            __syncthreads();
-        }
-        if (tid == 0) s_tot[l] = run;
-        __syncthreads();
-    }
-    // per step counts and their prefix (T is small: a serial loop in one thread)
-    if (tid == 0) {
-        long long acc = 0;
-        offsets[0] = 0;
-        for (int s = 0; s < c.T; ++s) {
-            bool d2, d1;
-            step_due(s, c, d2, d1);
-            acc += s_tot[2] + (d2 ? s_tot[1] : 0) + (d1 ? s_tot[0] : 0);
-            offsets[s + 1] = (int32_t)acc;
-        }
-    }
+// Due tokens of every step before step s, in closed form from the level
+// totals n1, n2, n3: each step lists Level 3; Level 2 when due2, Level 1 when
+// due1.  D(s, p) counts the steps s' < s in which a level of period p is due
+// (full steps count too).
+__device__ __forceinline__ long long due_before(int s, int p, const jano_sched_cfg& c) {
+    const int w = c.warmup, e = c.T - c.cooldown;        // interleaved steps are [w, e)
+    if (s <= w) return s;
+    const int si = min(s, e);
+    long long d = w + (si - w) / p;                      // j + 1 = 1 .. si - w, multiples of p
+    if (s > e) d += s - e;
+    return d;
+}
+
+__device__ __forceinline__ long long offset_of(int s, const jano_sched_cfg& c, const int (&tot)[3]) {
+    return (long long)s * tot[2] + due_before(s, c.period_moderate, c) * tot[1] +
+           due_before(s, c.period_static, c) * tot[0];
 }
 
 // The due set of a step is one of four unions of levels: {3}, {3,2}, {3,1},
-// {3,2,1} (set id = due2 | due1 << 1).  Each CTA ranks its tile's tokens in
-// all four once (ballots + one warp scan per set) and then writes the lists
-// of kStepsPerCta consecutive steps from those ranks.
-constexpr int kStepsPerCta = 8;
-
+// {3,2,1} (set id = due2 | due1 << 1).  One CTA per tile: it forms the
+// tile's per-level prefix over the earlier tiles and the level totals from
+// the count pass (a block reduction over the tile counts, no separate scan
+// launch), ranks the tile's tokens once in each of the four sets (ballots +
+// one warp scan per set) and stores the tile's part of every step's list;
+// the first CTA also writes offsets[].
 __global__ void __launch_bounds__(kTile)
 write_kernel(Ws ws, int n_tokens, int n_tiles, jano_sched_cfg c,
-             const int32_t* __restrict__ offsets, int32_t* __restrict__ idx) {
+             int32_t* __restrict__ offsets, int32_t* __restrict__ idx) {
     __shared__ int wc[4][32];
     __shared__ int wpre[4][32];
-    __shared__ int tpre[3];
+    __shared__ int red[6][32];
+    __shared__ int s_pre[3], s_tot[3];
+    constexpr int kStepChunk = 1024;
+    __shared__ long long s_base[kStepChunk];     // offsets of a chunk of steps
+    __shared__ unsigned char s_set[kStepChunk];  // their due sets
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tile = blockIdx.x;
+
+    // ---- per-level prefix over earlier tiles and totals over all tiles
+    int pre[3] = {0, 0, 0}, tot[3] = {0, 0, 0};
+    for (int i = tid; i < n_tiles; i += kTile) {
+#pragma unroll
+        for (int l = 0; l < 3; ++l) {
+            const int v = ws.cnt[l * n_tiles + i];
+            tot[l] += v;
+            if (i < tile) pre[l] += v;
+        }
+    }
+#pragma unroll
+    for (int l = 0; l < 3; ++l) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            pre[l] += __shfl_xor_sync(0xFFFFFFFFu, pre[l], o);
+            tot[l] += __shfl_xor_sync(0xFFFFFFFFu, tot[l], o);
+        }
+        if (lane == 0) { red[l][warp] = pre[l]; red[3 + l][warp] = tot[l]; }
+    }
+
+    // ---- ranks of the tile's tokens in the four due sets
     const int t = tile * kTile + tid;
     const int lv = t < n_tokens ? ws.tok[t] : 0;
     const unsigned lt = (1u << lane) - 1u;
@@ -167,27 +166,54 @@ write_kernel(Ws ws, int n_tokens, int n_tiles, jano_sched_cfg c,
         rank[set] = __popc(b & lt);
         if (lane == 0) wc[set][warp] = __popc(b);
     }
-    if (tid < 3) tpre[tid] = ws.pre[tid * n_tiles + tile];
     __syncthreads();
-    if (warp < 4) {
-        const int v = wc[warp][lane];
+    if (warp < 6) {
+        int v = red[warp][lane];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        if (lane == 0) {
+            if (warp < 3) s_pre[warp] = v;
+            else s_tot[warp - 3] = v;
+        }
+    } else if (warp < 10) {
+        const int set = warp - 6;
+        const int v = wc[set][lane];
         int incl = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
             if (lane >= o) incl += y;
         }
-        wpre[warp][lane] = incl - v;
+        wpre[set][lane] = incl - v;
     }
     __syncthreads();
-    const int s_end = min(c.T, (int)(blockIdx.y + 1) * kStepsPerCta);
-    for (int s = blockIdx.y * kStepsPerCta; s < s_end; ++s) {
-        bool d2, d1;
-        step_due(s, c, d2, d1);
-        const int set = (d2 ? 1 : 0) | (d1 ? 2 : 0);
-        if (in[set]) {
-            const long long base = (long long)offsets[s] + tpre[2] + (d2 ? tpre[1] : 0) + (d1 ? tpre[0] : 0);
-            idx[base + wpre[set][warp] + rank[set]] = t;
+    const int total[3] = {s_tot[0], s_tot[1], s_tot[2]};
+    // position of this token inside step lists of each set, less the step's offset
+    int pos[4];
+#pragma unroll
+    for (int set = 0; set < 4; ++set)
+        pos[set] = s_pre[2] + ((set & 1) ? s_pre[1] : 0) + ((set & 2) ? s_pre[0] : 0) +
+                   wpre[set][warp] + rank[set];
+    if (tile == 0 && tid == 0) offsets[0] = 0;
+
+    // ---- every step's part of this tile, steps staged in chunks
+    for (int s0 = 0; s0 < c.T; s0 += kStepChunk) {
+        const int ns = min(kStepChunk, c.T - s0);
+        __syncthreads();                     // the previous chunk's entries are consumed
+        if (tid < ns) {
+            const int s = s0 + tid;
+            bool d2, d1;
+            step_due(s, c, d2, d1);
+            s_set[tid] = (unsigned char)((d2 ? 1 : 0) | (d1 ? 2 : 0));
+            s_base[tid] = offset_of(s, c, total);
+            if (tile == 0) offsets[s + 1] = (int32_t)offset_of(s + 1, c, total);
+        }
+        __syncthreads();
+        for (int k = 0; k < ns; ++k) {
+            const int set = s_set[k];
+            const bool mine = set == 0 ? in[0] : set == 1 ? in[1] : set == 2 ? in[2] : in[3];
+            const int p = set == 0 ? pos[0] : set == 1 ? pos[1] : set == 2 ? pos[2] : pos[3];
+            if (mine) idx[s_base[k] + p] = t;
         }
     }
 }
@@ -208,7 +234,7 @@ Geo make_geo(const jano_geom& g) {
 size_t schedule_workspace_bytes(const jano_geom& g) {
     const long long nt = (long long)(g.F / g.pf) * (g.H / g.ph) * (g.W / g.pw);
     const long long tiles = (nt + kTile - 1) / kTile;
-    return align16((size_t)nt) + 2 * align16(sizeof(int) * 3 * (size_t)tiles);
+    return align16((size_t)nt) + align16(sizeof(int) * 3 * (size_t)tiles);
 }
 
 cudaError_t launch_build_schedule(const uint8_t* block_levels, const jano_geom& g,
@@ -221,9 +247,7 @@ cudaError_t launch_build_schedule(const uint8_t* block_levels, const jano_geom& 
     const Ws ws = carve(ws_base, n_tokens, n_tiles);
     count_kernel<<<n_tiles, kTile, 0, st>>>(block_levels, geo, n_tokens, token_levels, ws,
                                              n_tiles, err);
-    scan_kernel<<<1, kTile, 0, st>>>(ws, n_tiles, c, offsets);
-    write_kernel<<<dim3(n_tiles, (c.T + kStepsPerCta - 1) / kStepsPerCta), kTile, 0, st>>>(
-        ws, n_tokens, n_tiles, c, offsets, idx);
+    write_kernel<<<n_tiles, kTile, 0, st>>>(ws, n_tokens, n_tiles, c, offsets, idx);
     return cudaGetLastError();
 }
 

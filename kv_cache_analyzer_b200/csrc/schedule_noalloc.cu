@@ -22,9 +22,9 @@
 namespace jano {
 namespace {
 
-// 1 MiB: token levels (1 byte per token) plus two int32 [3][tiles] tables of
+// 1 MiB: token levels (1 byte per token) plus an int32 [3][tiles] table of
 // 1024-token tiles, each part rounded up to 16 bytes; that holds geometries
-// of at most 1,024,544 tokens (1,048,576 bytes exactly).
+// of at most 1,036,416 tokens (1,048,576 bytes exactly).
 constexpr size_t kStaticScratchBytes = size_t(1) << 20;
 
 static __device__ __align__(256) unsigned char g_schedule_scratch[kStaticScratchBytes];

@@ -45,8 +45,8 @@ def test_status_strings_and_version(jl):
 def test_workspace_query_is_host_only(jl):
     g = jl.Geometry(21, 90, 160, (1, 4, 4), (1, 2, 2))
     n = jl.jano_build_schedule_workspace_bytes(g.c())
-    # token levels (75600 B) + two int32 [3][74] tables, 16-byte rounded
-    assert n == 75600 + 2 * 896
+    # token levels (75600 B) + one int32 [3][74] table, 16-byte rounded
+    assert n == 75600 + 896
     bad = jl.Geometry(21, 91, 160, (1, 4, 4), (1, 2, 2))     # H not divisible by ph
     assert jl.jano_build_schedule_workspace_bytes(bad.c()) == 0
 
@@ -180,13 +180,13 @@ def test_split_choice_on_a_given_sm_count(jl):
 
 
 def test_noalloc_limit_is_exactly_its_scratch(jl):
-    # The static scratch is 1 MiB: align16(n) + 2 * align16(12 * ceil(n / 1024))
-    # bytes for n tokens.  317 x 3232 = 1,024,544 tokens need exactly 1 MiB;
-    # one token more (a 1 x 1,024,545 row) needs 1,048,592 bytes.
+    # The static scratch is 1 MiB: align16(n) + align16(12 * ceil(n / 1024))
+    # bytes for n tokens.  2699 x 384 = 1,036,416 tokens need exactly 1 MiB;
+    # one token more (a 1 x 1,036,417 row) needs 1,048,592 bytes.
     L = jl.lib()
-    at = jl.Geometry(1, 317, 3232, (1, 1, 1), (1, 1, 1))
-    over = jl.Geometry(1, 1, 1_024_545, (1, 1, 1), (1, 1, 1))
-    assert at.n_tokens == 1_024_544 and over.n_tokens == 1_024_545
+    at = jl.Geometry(1, 2699, 384, (1, 1, 1), (1, 1, 1))
+    over = jl.Geometry(1, 1, 1_036_417, (1, 1, 1), (1, 1, 1))
+    assert at.n_tokens == 1_036_416 and over.n_tokens == 1_036_417
     assert jl.jano_build_schedule_workspace_bytes(at.c()) == 1 << 20
     assert jl.jano_build_schedule_workspace_bytes(over.c()) == (1 << 20) + 16
     c = jl.Schedule(2, 1, 1, 1, 1).c()

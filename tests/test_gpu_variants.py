@@ -152,3 +152,19 @@ def test_fft_scores_edge_geometries(J, shape, block, cutoff):
     ref = oracle.fft_scores(x, block, cutoff)
     assert np.all(np.abs(got - ref) <= _fft_bound(x, block, ref))
     assert np.array_equal(got == 0, ref == 0)            # empty bands give exact zeros
+
+
+# ---------------------------------------------------------------- read-rate calibration
+@pytest.mark.parametrize("n,n_partial", [(4, 1), (1000, 7), (1 << 20, 148), (3_000_004, 148), (64, 148)])
+def test_stream_sum_partials(J, n, n_partial):
+    # jano_stream_sum (the one-pass read the analyzer's HBM rate is compared
+    # with): partial[i] is the fp32 sum of the i-th contiguous share of
+    # ceil(n/4 / n_partial) float4s; checked against fp64 sums of the same shares
+    g = np.random.default_rng(n)
+    x = g.standard_normal(n).astype(np.float32)
+    out = J.stream_sum(torch.from_numpy(x).cuda(), n_partial).cpu().numpy()
+    assert J.device_error() == 0
+    per = -(-(n // 4) // n_partial) * 4
+    ref = np.array([x[i * per:(i + 1) * per].astype(np.float64).sum() for i in range(n_partial)])
+    mag = np.array([np.abs(x[i * per:(i + 1) * per]).astype(np.float64).sum() for i in range(n_partial)])
+    assert np.all(np.abs(out - ref) <= 1e-5 * mag + 1e-6)

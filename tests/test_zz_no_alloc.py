@@ -78,8 +78,8 @@ def test_noalloc_schedule_matches_workspace_variant_on_two_calls(J):
 
 
 def test_noalloc_at_its_exact_limit_matches_workspace_variant(J):
-    # 317 x 3232 = 1,024,544 tokens fill the 1 MiB scratch exactly
-    g = J.Geometry(1, 317, 3232, (1, 4, 4), (1, 1, 1))
+    # 2699 x 384 = 1,036,416 tokens fill the 1 MiB scratch exactly
+    g = J.Geometry(1, 2699, 384, (1, 4, 4), (1, 1, 1))
     assert J.jano_build_schedule_workspace_bytes(g.c()) == 1 << 20
     lv = np.random.default_rng(3).integers(1, 4, size=g.n_blocks).astype(np.uint8)
     off = _run_both(J, lv, g, J.Schedule(3, 1, 1, 1, 1))
@@ -88,7 +88,7 @@ def test_noalloc_at_its_exact_limit_matches_workspace_variant(J):
 
 def test_noalloc_rejects_geometry_beyond_its_scratch(J):
     L = J.lib()
-    big = J.Geometry(1, 1, 1_024_545, (1, 1, 1), (1, 1, 1)).c()   # one token over the limit
+    big = J.Geometry(1, 1, 1_036_417, (1, 1, 1), (1, 1, 1)).c()   # one token over the limit
     c = J.Schedule(2, 1, 1, 1, 1).c()
     fake = C.c_void_p(256)
     assert L.jano_build_schedule_noalloc(fake, C.byref(big), C.byref(c), fake, fake, 10**9, None,
