@@ -64,6 +64,10 @@ constexpr int kRegsIssue = 80;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIssue <= kThreads * kRegsLaunch, "register split");
 static_assert(2 * kRegsSoftmax + kRegsIssue <= 512, "sub-partition register file");
 constexpr uint32_t kPanel = 128 * 128;   // bytes of one 128-row x 64-col BF16 panel
+// d = 128 and unsplit keys take the CTA-pair kernel when this is 1
+#ifndef JANO_ATTN_PAIR
+#define JANO_ATTN_PAIR 0
+#endif
 constexpr long long kWaitLimit = 1ll << 31;  // cycles (~1 s)
 
 template <int HD>
@@ -205,13 +209,7 @@ __device__ __forceinline__ float exp64(const uint32_t (&s)[64], int valid, float
         if (kMask && e >= valid) a = 0.f;
         if (kMask && e + 1 >= valid) b = 0.f;
         acc[(e >> 1) & 3] = ptx::fadd2(acc[(e >> 1) & 3], ptx::f2(a, b));
-#ifdef JANO_PACK_INT
-        // BF16 by integer rounding (half up; p >= 0 and finite), packed with
-        // one byte permute: keeps the conversion on the integer pipes
-        pk[e >> 1] = __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
-#else
         pk[e >> 1] = ptx::pack_bf16(a, b);
-#endif
     }
     const uint64_t t = ptx::fadd2(ptx::fadd2(acc[0], acc[1]), ptx::fadd2(acc[2], acc[3]));
     float lo, hi;
@@ -222,7 +220,9 @@ __device__ __forceinline__ float exp64(const uint32_t (&s)[64], int valid, float
 // One key tile of one query row: the row's 128 S values from TMEM in one
 // round trip, row max, lazy O rescale, P = 2^(S*c - m) as BF16 into the upper
 // half of the row's S columns.  Warp-uniform control flow throughout.
-template <int HD, bool kMask>
+// kRemote: bar_half is a shared::cluster address (the pair form's barriers
+// live in the even CTA) and is arrived on at cluster scope.
+template <int HD, bool kMask, bool kRemote = false>
 __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, uint32_t tP, int j, int valid,
                                              float c, float& m, float& l, uint32_t bar_half) {
     uint32_t s[128];
@@ -270,7 +270,10 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, uint32_t 
     ptx::tmem_wait_st();
     ptx::tc_fence_before();
     __syncwarp();
-    if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(bar_half);
+    if ((threadIdx.x & 31) == 0) {
+        if constexpr (kRemote) ptx::mbar_arrive_cluster(bar_half);
+        else ptx::mbar_arrive(bar_half);
+    }
     l += exp64<kMask>(lo, valid, c, m, pk);
     ptx::tmem_st32(tP, *reinterpret_cast<uint32_t(*)[32]>(pk));
     ptx::tmem_wait_st();
@@ -596,6 +599,360 @@ attention_combine_kernel(const float* __restrict__ part_o, const float2* __restr
     }
 }
 
+// ---------------------------------------------------------------------------
+// CTA-pair form (d = 128, keys not split).  A cluster of two CTAs on two SMs
+// takes four 128-query tiles of one head, two per CTA as above, and runs the
+// MMAs of both CTAs as pair MMAs (M = 256: query rows 0-127 from the even
+// CTA's shared memory and tensor memory, 128-255 from the odd CTA's), issued
+// by one thread of the even CTA.  The B operand of a pair MMA is split by N
+// between the two CTAs, so each CTA stages only half of every key tile: for
+// S = Q K^T keys [64 r, 64 r + 64) of the tile (all 128 columns), for
+// O += P V columns [64 r, 64 r + 64) of V (all 128 keys), r = the CTA's rank.
+// Per key tile an SM therefore receives 32 KB instead of 64 KB, and its
+// shared-memory port moves about 160 KB instead of 256 KB.  Every load is a
+// plain TMA load into the loading CTA's own shared memory (no multicast).
+//
+// Hand-offs between the two CTAs:
+//   - each CTA's copies complete on its own "landed" barriers; a relay thread
+//     of each CTA then arrives (cluster scope) on the even CTA's "full"
+//     barrier (2 arrivals: one per CTA), which the MMA thread waits on;
+//   - softmax warps of both CTAs publish P on the even CTA's P barriers
+//     (8 warp arrivals);
+//   - the MMA thread's commits are multicast to both CTAs (S ready, O ready,
+//     ring slot free, all MMAs done);
+//   - a CTA that gives up on a wait sets its own abort flag and the peer's;
+//   - tensor memory is allocated and freed at the same columns in both CTAs,
+//     and a cluster barrier ends the kernel, so neither CTA leaves while the
+//     pair's MMAs or the peer's remote arrivals may still touch it.
+// Every mbarrier wait is bounded.
+constexpr int kPairSlots = 8;                 // ring of K/V half tiles
+constexpr uint32_t kHalfTile = 16384;         // one K or V half tile (BF16)
+constexpr uint32_t kHalfPanel = 8192;         // 64 rows x 128 bytes
+
+struct PairLayout {
+    static constexpr uint32_t kQ0 = 0;
+    static constexpr uint32_t kQ1 = 2 * kPanel;
+    static constexpr uint32_t kRing = 4 * kPanel;
+    static constexpr uint32_t kBar = kRing + kPairSlots * kHalfTile;
+    static constexpr int bQLand = 0;                        // own Q tiles landed (tx)
+    static constexpr int bQFull = 1;                        // even CTA: both relays
+    static constexpr int bLand = 2;                         // [kPairSlots] own half landed (tx)
+    static constexpr int bFull = bLand + kPairSlots;        // [kPairSlots] even CTA: both relays
+    static constexpr int bEmpty = bFull + kPairSlots;       // [kPairSlots] commit, both CTAs
+    static constexpr int bSFull = bEmpty + kPairSlots;      // [2]
+    static constexpr int bPFull = bSFull + 2;               // [2] even CTA: 8 warp arrivals
+    static constexpr int bPHalf = bPFull + 2;               // [2] even CTA: 8 warp arrivals
+    static constexpr int bOFull = bPHalf + 2;               // [2]
+    static constexpr int bFinal = bOFull + 2;
+    static constexpr int kNumBars = bFinal + 1;
+    static constexpr uint32_t kMisc = kBar + 8 * kNumBars;  // tmem base, abort flag
+    static constexpr uint32_t kBytes = kMisc + 16;
+    static constexpr uint32_t kAlloc = kBytes + 1024;
+    static_assert(kAlloc <= 227 * 1024, "shared memory budget");
+};
+
+struct PairCtl {
+    uint32_t bar0;           // local address of barrier 0
+    uint32_t lead_bar0;      // shared::cluster address of barrier 0 in the even CTA
+    uint32_t peer_abort;     // shared::cluster address of the peer's abort flag
+    volatile int* abort;
+    int* err;
+    __device__ uint32_t bar(int i) const { return bar0 + 8u * (uint32_t)i; }
+    __device__ uint32_t lead(int i) const { return lead_bar0 + 8u * (uint32_t)i; }
+    __device__ void give_up() const {
+        *abort = 1;
+        ptx::st_cluster_u32(peer_abort, 1u);
+        raise_error(err, JANO_ETIMEOUT);
+    }
+    // Bounded wait with acquire at cluster scope (several barriers receive
+    // arrivals from the peer CTA or multicast commits); stops early once
+    // either CTA of the pair has given up.
+    __device__ bool wait(int i, uint32_t parity, bool spin = false) const {
+        auto poll = [&]() {
+            return spin ? ptx::mbar_try_wait_cluster(bar(i), parity)
+                        : ptx::mbar_try_wait_cluster_sleep(bar(i), parity);
+        };
+        if (poll()) return true;
+        const long long t0 = clock64();
+        for (;;) {
+            if (poll()) return true;
+            if (*abort) return false;
+            if (clock64() - t0 > kWaitLimit) {
+                give_up();
+                return false;
+            }
+        }
+    }
+    __device__ bool warp_wait(int i, uint32_t parity) const {
+        int ok = 0;
+        if ((threadIdx.x & 31) == 0) ok = wait(i, parity) ? 1 : 0;
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        return ok != 0;
+    }
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV,
+                      const int32_t* __restrict__ idx, int n_act, int n_tokens, int heads,
+                      float scale_log2, __nv_bfloat16* __restrict__ out, int* err) {
+    constexpr int HD = 128;
+    using L = PairLayout;
+    using LS = Layout<HD>;                      // TMEM columns as in the single-CTA form
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = ptx::smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = ptx::cluster_ctarank();
+    const bool lead = rank == 0;
+    const int head = blockIdx.y;
+    const int q0 = ((int)(blockIdx.x >> 1) * 4 + 2 * (int)rank) * BM;   // this CTA's tile 0
+    const int nt = (n_tokens + BN - 1) / BN;
+
+    PairCtl ctl;
+    ctl.bar0 = base + L::kBar;
+    ctl.lead_bar0 = ptx::mapa_shared(ctl.bar0, 0);
+    ctl.abort = reinterpret_cast<volatile int*>(gbase + L::kMisc + 4);
+    ctl.peer_abort = ptx::mapa_shared(base + L::kMisc + 4, rank ^ 1u);
+    ctl.err = err;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kMisc);
+
+    if (threadIdx.x == 0) {
+        ptx::prefetch_tmap(&tmQ);
+        ptx::prefetch_tmap(&tmK);
+        ptx::prefetch_tmap(&tmV);
+        ptx::mbar_init(ctl.bar(L::bQLand), 1);
+        ptx::mbar_init(ctl.bar(L::bQFull), 2);
+        for (int s = 0; s < kPairSlots; ++s) {
+            ptx::mbar_init(ctl.bar(L::bLand + s), 1);
+            ptx::mbar_init(ctl.bar(L::bFull + s), 2);
+            ptx::mbar_init(ctl.bar(L::bEmpty + s), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(ctl.bar(L::bSFull + i), 1);
+            ptx::mbar_init(ctl.bar(L::bPFull + i), 8);
+            ptx::mbar_init(ctl.bar(L::bPHalf + i), 8);
+            ptx::mbar_init(ctl.bar(L::bOFull + i), 1);
+        }
+        ptx::mbar_init(ctl.bar(L::bFinal), 1);
+        *ctl.abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 9) {
+        ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), 512);
+        ptx::tmem_relinquish_pair();
+    }
+    // both CTAs' barriers initialised and tensor memory allocated before any
+    // cross-CTA arrival or pair MMA
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync_all();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp >= 8) {
+      ptx::setmaxnreg_dec<kRegsIssue>();
+      if (warp == 8) {
+        // ------------------------------------------------------------ producer (each CTA)
+        if (lane == 0) {
+            int last[kPairSlots];
+            for (int s = 0; s < kPairSlots; ++s) last[s] = -1;
+            ptx::mbar_arrive_expect_tx(ctl.bar(L::bQLand), 4 * kPanel);
+            for (int p = 0; p < 2; ++p) {
+                ptx::tma_load_3d(base + L::kQ0 + p * kPanel, &tmQ, ctl.bar(L::bQLand), p * 64, head, q0);
+                ptx::tma_load_3d(base + L::kQ1 + p * kPanel, &tmQ, ctl.bar(L::bQLand), p * 64, head, q0 + BM);
+            }
+            // load n: K half (n even) or V half (n odd) of key tile n/2, into slot n % kPairSlots
+            for (int n = 0; n < 2 * nt; ++n) {
+                const int s = n % kPairSlots;
+                if (!ctl.wait(L::bEmpty + s, ((n / kPairSlots) & 1) ^ 1)) break;
+#ifdef JANO_INJECT_DROP_LOAD
+                if (n == JANO_INJECT_DROP_LOAD) continue;    // failure-path test builds only
+#endif
+                const uint32_t dst = base + L::kRing + s * kHalfTile;
+                const int kt = n >> 1;
+                ptx::mbar_arrive_expect_tx(ctl.bar(L::bLand + s), kHalfTile);
+                if ((n & 1) == 0) {
+                    // keys [64 r, 64 r + 64) of the tile, columns 0-63 and 64-127
+                    const int k0 = kt * BN + 64 * (int)rank;
+                    ptx::tma_load_3d(dst, &tmK, ctl.bar(L::bLand + s), 0, head, k0);
+                    ptx::tma_load_3d(dst + kHalfPanel, &tmK, ctl.bar(L::bLand + s), 64, head, k0);
+                } else {
+                    // columns [64 r, 64 r + 64) of V, keys 0-63 and 64-127 of the tile
+                    const int c0 = 64 * (int)rank;
+                    ptx::tma_load_3d(dst, &tmV, ctl.bar(L::bLand + s), c0, head, kt * BN);
+                    ptx::tma_load_3d(dst + kHalfPanel, &tmV, ctl.bar(L::bLand + s), c0, head, kt * BN + 64);
+                }
+                last[s] = n;
+            }
+            // drain: every copy this CTA issued lands before its smem is released
+            ptx::mbar_wait(ctl.bar(L::bQLand), 0, kWaitLimit);
+            for (int s = 0; s < kPairSlots; ++s)
+                if (last[s] >= 0) ptx::mbar_wait(ctl.bar(L::bLand + s), (last[s] / kPairSlots) & 1, kWaitLimit);
+        }
+      } else if (warp == 10) {
+        // ------------------------------------------------------------ relay (each CTA)
+        // this CTA's half of a stage has landed -> one arrival on the even CTA's full barrier
+        if (lane == 0 && ctl.wait(L::bQLand, 0)) {
+            ptx::mbar_arrive_cluster(ctl.lead(L::bQFull));
+            for (int n = 0; n < 2 * nt; ++n) {
+                const int s = n % kPairSlots;
+                if (!ctl.wait(L::bLand + s, (n / kPairSlots) & 1, true)) break;
+                ptx::mbar_arrive_cluster(ctl.lead(L::bFull + s));
+            }
+        }
+      } else if (warp == 9 && lead) {
+        // ------------------------------------------------------------ MMA issuer (even CTA)
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = ptx::idesc_bf16(2 * BM, BN, false, false);
+            constexpr uint32_t idesc_pv = ptx::idesc_bf16(2 * BM, HD, false, true);
+            constexpr uint16_t kBoth = 0x3;
+            auto slot_of = [](int n) { return n % kPairSlots; };
+            auto wait_full = [&](int n) { return ctl.wait(L::bFull + slot_of(n), (n / kPairSlots) & 1, true); };
+            auto commit = [&](int b) { ptx::mma_commit_pair_mc(ctl.bar(b), kBoth); };
+            auto qk = [&](int i, int n) {          // S_i = Q_i K^T, K halves in load n's slot
+                const uint32_t kb = base + L::kRing + slot_of(n) * kHalfTile;
+                const uint32_t qb = base + (i ? L::kQ1 : L::kQ0);
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    ptx::mma_ss_pair(tmem + LS::tS(i),
+                                     ptx::smem_desc_sw128(qb + (kk >> 2) * kPanel + (kk & 3) * 32, 16, 1024),
+                                     ptx::smem_desc_sw128(kb + (kk >> 2) * kHalfPanel + (kk & 3) * 32, 16, 1024),
+                                     idesc_qk, kk > 0 ? 1u : 0u);
+                }
+            };
+            // O_i += P_i V over key sixteenths [k0, k1); V halves in load n's slot
+            auto pv = [&](int i, int n, int k0, int k1, bool acc) {
+                const uint32_t vb = base + L::kRing + slot_of(n) * kHalfTile;
+#pragma unroll
+                for (int kk = k0; kk < k1; ++kk)
+                    ptx::mma_ts_pair(tmem + LS::tO(i), tmem + LS::tS(i) + LS::tP + kk * 8,
+                                     ptx::smem_desc_sw128(vb + kk * 2048, kHalfTile, 1024), idesc_pv,
+                                     (acc || kk > k0) ? 1u : 0u);
+            };
+            auto pv_tile = [&](int i, int n, int j) -> bool {
+                if (!ctl.wait(L::bPHalf + i, j & 1, true)) return false;
+                ptx::tc_fence_after();
+                pv(i, n, BN / 32, BN / 16, j > 0);
+                if (!ctl.wait(L::bPFull + i, j & 1, true)) return false;
+                ptx::tc_fence_after();
+                pv(i, n, 0, BN / 32, true);
+                return true;
+            };
+            bool ok = ctl.wait(L::bQFull, 0) && wait_full(0);
+            if (ok) {
+                ptx::tc_fence_after();
+                qk(0, 0);
+                commit(L::bSFull + 0);
+                qk(1, 0);
+                commit(L::bSFull + 1);
+                commit(L::bEmpty + slot_of(0));
+            }
+            for (int j = 1; ok && j < nt; ++j) {
+                const int nk = 2 * j, nv = 2 * j - 1;        // loads of K_j and V_{j-1}
+                if (!wait_full(nv) || !wait_full(nk)) { ok = false; break; }
+                ptx::tc_fence_after();
+                if (!pv_tile(0, nv, j - 1)) { ok = false; break; }
+                qk(0, nk);
+                commit(L::bSFull + 0);
+                if (!pv_tile(1, nv, j - 1)) { ok = false; break; }
+                commit(L::bEmpty + slot_of(nv));
+                qk(1, nk);
+                commit(L::bSFull + 1);
+                commit(L::bEmpty + slot_of(nk));
+            }
+            if (ok) {
+                const int nv = 2 * nt - 1;
+                ok = wait_full(nv);
+                if (ok) {
+                    ptx::tc_fence_after();
+                    ok = pv_tile(0, nv, nt - 1);
+                }
+                if (ok) {
+                    commit(L::bOFull + 0);
+                    ok = pv_tile(1, nv, nt - 1);
+                }
+                if (ok) {
+                    commit(L::bOFull + 1);
+                    commit(L::bEmpty + slot_of(nv));
+                }
+            }
+            // every pair MMA is complete (in both CTAs) before tensor memory is released
+            commit(L::bFinal);
+            ptx::mbar_wait(ctl.bar(L::bFinal), 0, kWaitLimit);
+        }
+      } else if (warp == 9) {
+        // odd CTA: the final commit's arrival has landed here before this CTA
+        // can leave (the even CTA commits it on every path, aborts included)
+        if (lane == 0) ptx::mbar_wait(ctl.bar(L::bFinal), 0, kWaitLimit);
+      }
+    } else {
+        ptx::setmaxnreg_inc<kRegsSoftmax>();
+        // ------------------------------------------------------------ softmax WG i (each CTA)
+        const int i = warp >> 2;
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        const uint32_t tS = tmem + lane_off + LS::tS(i);
+        const uint32_t tO = tmem + lane_off + LS::tO(i);
+        const int qi = q0 + i * BM + row;
+        int t_out = -1;
+        if (qi < n_act) {
+            t_out = __ldg(idx + qi);
+            if (t_out < 0 || t_out >= n_tokens || (qi > 0 && __ldg(idx + qi - 1) >= t_out)) {
+                raise_error(err, JANO_EINDEX);
+                t_out = -1;
+            }
+        }
+        float m = -INFINITY, l = 0.f;
+        const int tail = n_tokens - (nt - 1) * BN;
+        bool ok = true;
+        for (int j = 0; j < nt; ++j) {
+            if (!ctl.warp_wait(L::bSFull + i, j & 1)) { ok = false; break; }
+            ptx::tc_fence_after();
+            if (j < nt - 1 || tail == BN)
+                softmax_tile<HD, false, true>(tS, tO, tS + LS::tP, j, BN, scale_log2, m, l, ctl.lead(L::bPHalf + i));
+            else
+                softmax_tile<HD, true, true>(tS, tO, tS + LS::tP, j, tail, scale_log2, m, l, ctl.lead(L::bPHalf + i));
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_cluster(ctl.lead(L::bPFull + i));
+        }
+        if (ok && ctl.warp_wait(L::bOFull + i, 0)) {
+            ptx::tc_fence_after();
+            const float inv = 1.0f / l;
+            __nv_bfloat16* orow = out + ((size_t)(t_out < 0 ? 0 : t_out) * heads + head) * HD;
+#pragma unroll
+            for (int c = 0; c < HD / 32; ++c) {
+                uint32_t o[32];
+                ptx::tmem_ld32(tO + 32 * c, o);
+                ptx::tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = ptx::pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+                if (t_out >= 0) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                }
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    // neither CTA leaves (or frees its tensor memory) while the pair's MMAs or
+    // the peer's remote arrivals may still reach it
+    ptx::cluster_sync_all();
+    ptx::tc_fence_after();
+    if (warp == 9) ptx::tmem_dealloc_pair(tmem, 512);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -609,13 +966,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 3D map over [rows][heads][d] BF16, box = 64 columns x 1 head x 128 rows.
-bool make_map(CUtensorMap* m, const void* ptr, int rows, int heads, int d) {
+// 3D map over [rows][heads][d] BF16, box = 64 columns x 1 head x box_rows rows.
+bool make_map(CUtensorMap* m, const void* ptr, int rows, int heads, int d, int box_rows = 128) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
     const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2};
-    const cuuint32_t box[3] = {64, 1, 128};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
     const cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -661,6 +1018,35 @@ cudaError_t launch_hd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
     const long long rows = (long long)n_act * heads;
     attention_combine_kernel<HD><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
         part_o, part_ml, idx, n_act, n_tokens, heads, n_split, static_cast<__nv_bfloat16*>(out), err);
+    return cudaGetLastError();
+}
+
+// The CTA-pair kernel (d = 128, keys not split): clusters of two CTAs, four
+// query tiles per cluster.
+cudaError_t launch_pair(const void* q, const void* k, const void* v, const int32_t* idx, int n_act,
+                        int n_tokens, int heads, float scale, void* out, int* err, cudaStream_t st) {
+    static DeviceOnce ready;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!ready.done(dev)) {
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, attention_pair_kernel);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
+        e = cudaFuncSetAttribute(attention_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)PairLayout::kAlloc);
+        if (e != cudaSuccess) return e;
+        ready.mark(dev);
+    }
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, n_act, heads, 128, 128) || !make_map(&mk, k, n_tokens, heads, 128, 64) ||
+        !make_map(&mv, v, n_tokens, heads, 128, 64))
+        return cudaErrorInvalidValue;
+    const int q_tiles = (n_act + BM - 1) / BM;
+    const dim3 grid(2 * ((q_tiles + 3) / 4), heads, 1);
+    attention_pair_kernel<<<grid, kThreads, PairLayout::kAlloc, st>>>(
+        mq, mk, mv, idx, n_act, n_tokens, heads, scale * 1.4426950408889634f,
+        static_cast<__nv_bfloat16*>(out), err);
     return cudaGetLastError();
 }
 
@@ -711,6 +1097,10 @@ cudaError_t launch_active_attention(const void* q, const void* k, const void* v,
                                     int heads, int d, float scale, void* out,
                                     int* err, cudaStream_t st, int n_split, void* ws) {
     if (n_act <= 0) return cudaSuccess;
+#if JANO_ATTN_PAIR
+    if (d == 128 && n_split == 1)
+        return launch_pair(q, k, v, idx, n_act, n_tokens, heads, scale, out, err, st);
+#endif
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, n_act, heads, d) || !make_map(&mk, k, n_tokens, heads, d) ||
         !make_map(&mv, v, n_tokens, heads, d))
