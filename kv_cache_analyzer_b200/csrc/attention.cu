@@ -504,10 +504,12 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
                     for (int e = 0; e < 16; ++e)
                         pk[e] = ptx::pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
                     if (t_out >= 0) {
+                        // streaming stores: the output rows are not read again here,
+                        // so they should leave L2 early rather than linger dirty
                         uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
                         for (int v = 0; v < 4; ++v)
-                            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                            __stcs(dst + v, make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]));
                     }
                 }
             } else {
@@ -664,13 +666,16 @@ struct PairCtl {
         ptx::st_cluster_u32(peer_abort, 1u);
         raise_error(err, JANO_ETIMEOUT);
     }
-    // Bounded wait with acquire at cluster scope (several barriers receive
-    // arrivals from the peer CTA or multicast commits); stops early once
-    // either CTA of the pair has given up.
-    __device__ bool wait(int i, uint32_t parity, bool spin = false) const {
+    // Bounded wait; stops early once either CTA of the pair has given up.
+    // cluster: acquire at cluster scope, for the barriers that other CTAs'
+    // threads arrive on (the even CTA's full and P barriers); the others only
+    // receive this CTA's arrivals, its copies and tensor-core commits.
+    __device__ bool wait(int i, uint32_t parity, bool spin = false, bool cluster = false) const {
         auto poll = [&]() {
-            return spin ? ptx::mbar_try_wait_cluster(bar(i), parity)
-                        : ptx::mbar_try_wait_cluster_sleep(bar(i), parity);
+            if (cluster)
+                return spin ? ptx::mbar_try_wait_cluster(bar(i), parity)
+                            : ptx::mbar_try_wait_cluster_sleep(bar(i), parity);
+            return spin ? ptx::mbar_try_wait(bar(i), parity) : ptx::mbar_try_wait_sleep(bar(i), parity);
         };
         if (poll()) return true;
         const long long t0 = clock64();
@@ -811,7 +816,7 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
             constexpr uint32_t idesc_pv = ptx::idesc_bf16(2 * BM, HD, false, true);
             constexpr uint16_t kBoth = 0x3;
             auto slot_of = [](int n) { return n % kPairSlots; };
-            auto wait_full = [&](int n) { return ctl.wait(L::bFull + slot_of(n), (n / kPairSlots) & 1, true); };
+            auto wait_full = [&](int n) { return ctl.wait(L::bFull + slot_of(n), (n / kPairSlots) & 1, true, true); };
             auto commit = [&](int b) { ptx::mma_commit_pair_mc(ctl.bar(b), kBoth); };
             auto qk = [&](int i, int n) {          // S_i = Q_i K^T, K halves in load n's slot
                 const uint32_t kb = base + L::kRing + slot_of(n) * kHalfTile;
@@ -834,15 +839,15 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
                                      (acc || kk > k0) ? 1u : 0u);
             };
             auto pv_tile = [&](int i, int n, int j) -> bool {
-                if (!ctl.wait(L::bPHalf + i, j & 1, true)) return false;
+                if (!ctl.wait(L::bPHalf + i, j & 1, true, true)) return false;
                 ptx::tc_fence_after();
                 pv(i, n, BN / 32, BN / 16, j > 0);
-                if (!ctl.wait(L::bPFull + i, j & 1, true)) return false;
+                if (!ctl.wait(L::bPFull + i, j & 1, true, true)) return false;
                 ptx::tc_fence_after();
                 pv(i, n, 0, BN / 32, true);
                 return true;
             };
-            bool ok = ctl.wait(L::bQFull, 0) && wait_full(0);
+            bool ok = ctl.wait(L::bQFull, 0, false, true) && wait_full(0);
             if (ok) {
                 ptx::tc_fence_after();
                 qk(0, 0);
@@ -938,7 +943,7 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
                     uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
                     for (int v = 0; v < 4; ++v)
-                        dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                        __stcs(dst + v, make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]));
                 }
             }
         }

@@ -6,18 +6,25 @@
 // its rank is below k_static = n_S and Active when its rank is at least
 // k_active = n - n_A.  Instead of sorting, the kernel finds, for each of the
 // two rank thresholds, the 32-bit order-preserving score key at that rank by
-// an MSB-first radix select (digits of 11, 11 and 10 bits), then resolves
-// ties at the threshold value by block index in one pass in index order.
+// a most-significant-first radix select, then resolves ties at the threshold
+// value by block index in one pass in index order.
+//
+// The select works on the range of keys that occur, [min, max]: each pass
+// splits the current bucket of both targets into 2048 bins of 2^shift keys
+// (the first bucket is the whole range, so the bins spread over the keys
+// present and shared-memory atomics rarely collide), keeps the bin holding
+// the target rank, and stops once a bin is a single key (at most three
+// passes for 32-bit keys, one when all keys are equal).
 //
 // One thread-block cluster of 8 CTAs does the work with no global scratch:
-// each CTA histograms its eighth of the scores in shared memory (warp-
-// aggregated atomics, since most keys share their top digits; the first pass,
-// which has no prefix yet, builds one histogram for both targets), the 8
+// each CTA histograms its eighth of the scores in shared memory (plain
+// atomics; the first pass builds one histogram for both targets), the 8
 // histograms are summed through distributed shared memory after a cluster
 // barrier (each thread issues all its remote loads before using any), and
-// every CTA finds the same digit by a block-wide scan of the totals (two
-// bins per thread).  Histograms are double buffered so one cluster barrier
-// per pass suffices.  The tie pass counts
+// every CTA finds the same bin by a block-wide scan of the totals (two bins
+// per thread).  Histograms are double buffered so one cluster barrier per
+// pass suffices.  The key range and the non-finite check ride on the first
+// cluster barrier.  The tie pass counts
 // threshold ties per thread over a contiguous range, scans them inside the
 // CTA and across the 8 CTAs (again through distributed shared memory), then
 // writes the levels.  Each CTA keeps its slice of keys in shared memory
@@ -34,11 +41,9 @@ namespace {
 
 constexpr int kCluster = 8;
 constexpr int kThreads = 1024;
-constexpr int kBins = 2048;             // 11-bit digits
-constexpr int kPasses = 3;
+constexpr int kBinBits = 11;
+constexpr int kBins = 1 << kBinBits;    // bins per histogram
 constexpr int kMaxCachedKeys = 40 * 1024;   // keys per CTA kept in shared memory (160 KB)
-__host__ __device__ constexpr int digit_shift(int pass) { return pass == 0 ? 21 : (pass == 1 ? 10 : 0); }
-__host__ __device__ constexpr int digit_width(int pass) { return pass == 2 ? 10 : 11; }
 
 // Order-preserving map float bits -> uint32 (unsigned order == float order),
 // with -0 folded onto +0.
@@ -52,17 +57,15 @@ struct Shared {
     // the pass's cluster barrier has passed, no peer reads buffer (p&1)^1 any
     // more, so it holds this CTA's copy of the cluster-wide totals.
     unsigned hist[2][2][kBins];
-    unsigned val[2], need[2];            // per target: key prefix, rank left
+    unsigned lo[2], need[2];             // per target: bucket start (key), rank left in it
     unsigned wsum[2][32];
     unsigned ctot[2];                    // this CTA's tie counts (read by peers)
+    unsigned kmin, kmax;                 // this CTA's key range (read by peers)
     int bad;
 };
 
-__device__ __forceinline__ void warp_agg_add(unsigned* h, unsigned active, unsigned dg, bool mine) {
-    if (!mine) return;
-    const unsigned peers = __match_any_sync(active, dg);
-    if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[dg], __popc(peers));
-}
+// Bits needed to write x (0 for x == 0).
+__device__ __forceinline__ int bit_length(uint32_t x) { return x ? 32 - __clz(x) : 0; }
 
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
 classify_kernel(const uint32_t* __restrict__ bits, int n, long long k_static,
@@ -80,59 +83,74 @@ classify_kernel(const uint32_t* __restrict__ bits, int n, long long k_static,
     const bool live0 = k_static > 0 && k_static < n;
     const bool live1 = k_active > 0 && k_active < n;
 
-    // ---- one coalesced sweep: non-finite check, keys into shared memory
+    // ---- one coalesced sweep: non-finite check, key range, keys into shared memory
     const bool use_cache = hi - lo <= kMaxCachedKeys;
     int bad = 0;
+    uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
     for (int i = lo + tid; i < hi; i += kThreads) {
         const uint32_t b = __ldg(bits + i);
         bad |= (b & 0x7F800000u) == 0x7F800000u;
-        if (use_cache) cached[i - lo] = order_key(b);
+        const uint32_t u = order_key(b);
+        kmn = min(kmn, u);
+        kmx = max(kmx, u);
+        if (use_cache) cached[i - lo] = u;
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        kmn = min(kmn, __shfl_xor_sync(0xFFFFFFFFu, kmn, o));
+        kmx = max(kmx, __shfl_xor_sync(0xFFFFFFFFu, kmx, o));
+    }
+    if (tid == 0) { sh.kmin = 0xFFFFFFFFu; sh.kmax = 0u; }
+    __syncthreads();
+    if (lane == 0) { atomicMin(&sh.kmin, kmn); atomicMax(&sh.kmax, kmx); }
     bad = __syncthreads_or(bad);
     // key of element i (lo <= i < hi)
     auto key = [&](int i) { return use_cache ? cached[i - lo] : order_key(__ldg(bits + i)); };
     if (tid == 0) {
         sh.bad = bad;
-        sh.val[0] = sh.val[1] = 0u;
         sh.need[0] = (unsigned)(k_static < 0 ? 0 : (k_static > n ? n : k_static));
         sh.need[1] = (unsigned)(k_active < 0 ? 0 : (k_active > n ? n : k_active));
     }
     cluster.sync();
     int any_bad = 0;
-    for (int r = 0; r < kCluster; ++r) any_bad |= *cluster.map_shared_rank(&sh.bad, r);
+    uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
+    for (int r = 0; r < kCluster; ++r) {
+        const Shared* peer = cluster.map_shared_rank(&sh, r);
+        any_bad |= peer->bad;
+        gmin = min(gmin, peer->kmin);
+        gmax = max(gmax, peer->kmax);
+    }
     if (any_bad) {
         if (rank == 0 && tid == 0) raise_error(err, JANO_ENONFINITE);
-        cluster.sync();            // peers may still be reading our flag
+        cluster.sync();            // peers may still be reading our flags
         return;
     }
 
-    // ---- radix select, most significant digit first
-    for (int pass = 0; pass < kPasses; ++pass) {
-        const int buf = pass & 1, shift = digit_shift(pass);
-        const unsigned dmask = (1u << digit_width(pass)) - 1u;
-        const uint32_t hmask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + digit_width(pass)));
-        // pass 0 has no prefix yet: one histogram serves both targets
-        const bool one = pass == 0;
+    // ---- radix select over the key range [gmin, gmax], most significant digit
+    // first.  Each pass splits the current bucket of both targets into 2048
+    // bins of 2^shift keys; the first pass's bucket is the whole range (so the
+    // bins spread over the keys that occur, which keeps atomics apart), and
+    // the passes stop once a bin is a single key.
+    int shift = max(0, bit_length(gmax - gmin) - kBinBits);
+    int bucket_bits = 32;                    // width of the current buckets, log2
+    if (tid == 0) sh.lo[0] = sh.lo[1] = gmin;
+    for (int pass = 0;; ++pass) {
+        const int buf = pass & 1;
+        const bool one = pass == 0;          // one histogram serves both targets
         const int nh = one ? 1 : 2;
         for (int b = tid; b < nh * kBins; b += kThreads) (&sh.hist[buf][0][0])[b] = 0u;
-        const uint32_t p0 = sh.val[0] & hmask, p1 = sh.val[1] & hmask;
+        __syncthreads();                     // sh.lo of the previous pass is visible too
+        const uint32_t lo0 = sh.lo[0], lo1 = sh.lo[1];
         const unsigned need0 = sh.need[0], need1 = sh.need[1];
-        __syncthreads();
-        for (int base = lo; base < hi; base += kThreads) {
-            const int i = base + tid;
-            const bool ok = i < hi;
-            const uint32_t u = ok ? key(i) : 0u;
-            const unsigned dg = (u >> shift) & dmask;
+        // candidates: keys inside the target's current bucket of 2^bucket_bits keys
+        const uint32_t width_m1 = bucket_bits >= 32 ? 0xFFFFFFFFu : (1u << bucket_bits) - 1u;
+        for (int i = lo + tid; i < hi; i += kThreads) {
+            const uint32_t u = key(i);
             if (one) {
-                const bool m = ok && (live0 || live1);
-                warp_agg_add(sh.hist[buf][0], __ballot_sync(0xFFFFFFFFu, m), dg, m);
+                if (live0 || live1) atomicAdd(&sh.hist[buf][0][(u - lo0) >> shift], 1u);
             } else {
-                const bool m0 = ok && live0 && (u & hmask) == p0;
-                const bool m1 = ok && live1 && (u & hmask) == p1;
-                const unsigned a0 = __ballot_sync(0xFFFFFFFFu, m0);
-                const unsigned a1 = __ballot_sync(0xFFFFFFFFu, m1);
-                warp_agg_add(sh.hist[buf][0], a0, dg, m0);
-                warp_agg_add(sh.hist[buf][1], a1, dg, m1);
+                if (live0 && u - lo0 <= width_m1) atomicAdd(&sh.hist[buf][0][(u - lo0) >> shift], 1u);
+                if (live1 && u - lo1 <= width_m1) atomicAdd(&sh.hist[buf][1][(u - lo1) >> shift], 1u);
             }
         }
         cluster.sync();            // all 8 local histograms of this pass are complete
@@ -187,23 +205,26 @@ classify_kernel(const uint32_t* __restrict__ bits, int n, long long k_static,
             sh.wsum[1][lane] = j1 - w1;
         }
         __syncthreads();
-        // the one thread whose two bins hold rank `need` fixes the digit
+        // the one thread whose two bins hold rank `need` narrows the bucket
         const unsigned e0 = sh.wsum[0][warp] + i0 - x0, e1 = sh.wsum[1][warp] + i1 - x1;
         if (live0 && e0 <= need0 && need0 < e0 + x0) {
             const bool first = need0 < e0 + a0;
-            sh.val[0] |= (uint32_t)(2 * tid + (first ? 0 : 1)) << shift;
+            sh.lo[0] = lo0 + ((uint32_t)(2 * tid + (first ? 0 : 1)) << shift);
             sh.need[0] = need0 - e0 - (first ? 0u : a0);
         }
         if (live1 && e1 <= need1 && need1 < e1 + x1) {
             const bool first = need1 < e1 + a1;
-            sh.val[1] |= (uint32_t)(2 * tid + (first ? 0 : 1)) << shift;
+            sh.lo[1] = lo1 + ((uint32_t)(2 * tid + (first ? 0 : 1)) << shift);
             sh.need[1] = need1 - e1 - (first ? 0u : a1);
         }
-        __syncthreads();
+        if (shift == 0) break;              // the bucket is one key: its value is lo
+        bucket_bits = shift;
+        shift = max(0, shift - kBinBits);
     }
+    __syncthreads();
 
     // ---- ties at the threshold values, resolved by block index
-    const uint32_t v0 = sh.val[0], v1 = sh.val[1];
+    const uint32_t v0 = sh.lo[0], v1 = sh.lo[1];
     const unsigned need0 = sh.need[0], need1 = sh.need[1];
     const int per_thr = (hi - lo + kThreads - 1) / kThreads;
     const int tlo = min(hi, lo + tid * per_thr), thi = min(hi, tlo + per_thr);
