@@ -77,7 +77,12 @@ def test_block_scores_match_oracle(J, name):
                                          ((6, 1, 1, 16, 16), (1, 2, 2)),    # F = 1
                                          ((3, 1, 2, 4, 20), (1, 4, 8)),     # bw = 8, partial
                                          ((4, 3, 3, 9, 520), (1, 4, 4)),    # wide rows: boxed chunks
-                                         ((3, 2, 2, 6, 200), (2, 4, 8))])   # whole rows, bf = 2
+                                         ((3, 2, 2, 6, 200), (2, 4, 8)),    # whole rows, bf = 2
+                                         # K = 5 with 1x4x4 blocks (the frame-run path):
+                                         ((6, 2, 1, 9, 20), (1, 4, 4)),     # F = 1, partial row, odd blocks
+                                         ((6, 3, 5, 14, 200), (1, 4, 4)),   # two column chunks, ragged
+                                         ((6, 2, 11, 8, 328), (1, 4, 4)),   # runs of several frames
+                                         ((6, 1, 21, 6, 48), (1, 4, 4))])   # many runs, short rows
 def test_block_scores_edge_geometries(J, shape, block):
     g = np.random.default_rng(sum(shape))
     lat = g.standard_normal(shape).astype(np.float32)
