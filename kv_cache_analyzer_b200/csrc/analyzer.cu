@@ -31,6 +31,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "jano_common.cuh"
@@ -289,6 +291,181 @@ analyzer_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
 }
 
+// ---------------------------------------------------------------------------
+// Frame-group form: the default reading with K = 5 and blocks of one frame,
+// at most 4 rows (1, 2 or 4) and 1-32 columns (a power of two) -- every
+// workload of the pages' configurations.  A work unit is G consecutive
+// frames x 4 rows x Wc columns (Wc a multiple of 32); its stage per channel
+// is box A (all K+1 snapshots of the G frames, the 4 rows and the h+1 halo
+// row, Wc + 4 columns) and box B (the frame after the group, 4 rows,
+// snapshots 1..K-1).  Only the group's last frame takes its f+1 neighbour
+// from box B; the others find it in box A, so the bytes each stage brings
+// from L2 per frame fall with G (on the large video latent: 177 MB for the
+// 116 MB read once from HBM, against 235 MB with one frame per unit).
+// Warp = one frame x 4 rows x 32 columns, lane = (row, float4), so a
+// quarter-warp reads 128 consecutive bytes of one staged row.  Each thread
+// evaluates all K-1 steps of its 4 columns per stage (its K+1 snapshots in
+// registers, the neighbours read as each step needs them) and the warp
+// frees the slot after the arithmetic; at 64 registers a thread, several
+// small CTAs share an SM, each with a short ring of its own.  At the end of a unit
+// the block sums are formed by warp shuffles (xor butterflies over the rows
+// of a block and, for blocks wider than 4 columns, over its float4 lanes):
+// each partner pair adds the same two values, so every lane of a block ends
+// with the same bits whatever the scheduling (deterministic).
+struct FGeo {
+    int C, F, H, W;
+    int bh, bw, nBh, nBw;
+    int G, Wc, LA;                 // frames and columns per unit, staged row length (Wc + 4)
+    int n_wc, n_rg, n_units;       // units along W, row groups of 4 along H, all units
+    int n_warps;                   // compute warps: G x Wc / 32
+    int S, stage_bytes, bytesA, bytesB, offB, smem;
+    float w_t, w_s;
+};
+
+#ifndef JANO_ANALYZER_FG
+#define JANO_ANALYZER_FG 1
+#endif
+constexpr int kFgMaxThreads = 512;
+
+template <int K>
+__global__ void __launch_bounds__(kFgMaxThreads)
+analyzer_fg_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   FGeo g, float* __restrict__ scores, int* err) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = ptx::smem_u32(smem_raw);
+    const uint32_t base = (raw + 127u) & ~127u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    const int S = g.S;
+    const uint32_t bars = base + (uint32_t)(S * g.stage_bytes);        // S full, S empty barriers
+    volatile int* abort = reinterpret_cast<volatile int*>(gbase + S * g.stage_bytes + 16 * S);
+    auto full = [&](int s) { return bars + 8u * s; };
+    auto empty = [&](int s) { return bars + 8u * (S + s); };
+    const int n_compute = g.n_warps * 32;
+
+    if (threadIdx.x == 0) {
+        ptx::prefetch_tmap(&tmA);
+        ptx::prefetch_tmap(&tmB);
+        for (int s = 0; s < S; ++s) {
+            ptx::mbar_init(full(s), 1);
+            ptx::mbar_init(empty(s), g.n_warps);
+        }
+        *abort = 0;
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+
+    const int tid = threadIdx.x;
+    if (tid >= n_compute) {
+        // ------------------------------------------------------------ producer
+        if (tid == n_compute) {
+            int last[kMaxStages];                 // phase of the last copy into each slot
+            for (int q = 0; q < S; ++q) last[q] = -1;
+            int slot = 0, phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < g.n_units; u += gridDim.x) {
+                const int wc = u % g.n_wc;
+                const int rg = (u / g.n_wc) % g.n_rg;
+                const int fg = u / (g.n_wc * g.n_rg);
+                const int f0 = fg * g.G, h0 = rg * 4, w0 = wc * g.Wc;
+                const bool has_next = f0 + g.G < g.F;
+                for (int c = 0; c < g.C; ++c) {
+                    if (!bounded_wait(empty(slot), (uint32_t)(phase ^ 1), err, abort)) { ok = false; break; }
+                    const uint32_t dst = base + (uint32_t)slot * g.stage_bytes;
+                    ptx::mbar_arrive_expect_tx(full(slot), g.bytesA + (has_next ? g.bytesB : 0));
+                    tma_load_5d(dst, &tmA, full(slot), w0, h0, f0, c, 0);
+                    if (has_next) tma_load_5d(dst + g.offB, &tmB, full(slot), w0, h0, f0 + g.G, c, 1);
+                    last[slot] = phase;
+                    if (++slot == S) { slot = 0; phase ^= 1; }
+                }
+            }
+            for (int q = 0; q < S; ++q)
+                if (last[q] >= 0) ptx::mbar_wait(full(q), (uint32_t)last[q], kWaitLimit);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- compute
+    const int warp = tid >> 5, lane = tid & 31;
+    const int wpf = g.Wc >> 5;                         // warps per frame
+    const int fr = warp / wpf;                         // frame inside the group
+    const int hr = lane >> 3;                          // row inside the unit
+    const int wr = ((warp % wpf) << 5) + ((lane & 7) << 2);   // first column inside the unit
+    const int LA = g.LA;
+    // float offsets inside a stage: this row at snapshot 0, the snapshot
+    // stride of box A, and the f+1 neighbour (box A, or box B for the
+    // group's last frame) as base + k * stride for snapshot k
+    const int oA = (fr * 5 + hr) * LA + wr;
+    const int sA = g.G * 5 * LA;
+    const bool nf_in_A = fr + 1 < g.G;
+    const int oF = nf_in_A ? oA + 5 * LA : g.offB / 4 + hr * g.Wc + wr - 4 * g.Wc;
+    const int sF = nf_in_A ? sA : 4 * g.Wc;
+    const float w_t = g.w_t, w_s = g.w_s;
+    int slot = 0, phase = 0;
+    for (int u = blockIdx.x; u < g.n_units; u += gridDim.x) {
+        const int wc = u % g.n_wc;
+        const int rg = (u / g.n_wc) % g.n_rg;
+        const int fg = u / (g.n_wc * g.n_rg);
+        const int f = fg * g.G + fr, h = rg * 4 + hr, w = wc * g.Wc + wr;
+        const bool act = f < g.F && h < g.H && w < g.W;      // W is a multiple of 4
+        const bool has_f = f + 1 < g.F, has_h = h + 1 < g.H, has_w = w + 4 < g.W;
+        // a warp whose lanes all have every neighbour takes the unmasked path
+        const bool interior = __all_sync(0xFFFFFFFFu, act && has_f && has_h && has_w);
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        for (int c = 0; c < g.C; ++c) {
+            const bool ready = bounded_wait(full(slot), (uint32_t)phase, err, abort);
+            if (ready && act) {
+                const float* A = reinterpret_cast<const float*>(gbase + (size_t)slot * g.stage_bytes);
+                float4 x[K + 1];
+#pragma unroll
+                for (int s = 0; s <= K; ++s) x[s] = *reinterpret_cast<const float4*>(A + oA + s * sA);
+#pragma unroll
+                for (int k = 1; k < K; ++k) {
+                    const float4 xm = x[k - 1], x0 = x[k], xp = x[k + 1];
+                    float4 nhk = *reinterpret_cast<const float4*>(A + oA + k * sA + LA);
+                    float4 nfk = *reinterpret_cast<const float4*>(A + oF + k * sF);
+                    float nxk = A[oA + k * sA + 4];
+                    if (!interior) {
+                        if (!has_h) nhk = x0;
+                        if (!has_f) nfk = x0;
+                        if (!has_w) nxk = x0.w;
+                    }
+                    a0 += term(xp.x - 2.f * x0.x + xm.x, nfk.x - x0.x, nhk.x - x0.x, x0.y - x0.x, w_t, w_s);
+                    a1 += term(xp.y - 2.f * x0.y + xm.y, nfk.y - x0.y, nhk.y - x0.y, x0.z - x0.y, w_t, w_s);
+                    a2 += term(xp.z - 2.f * x0.z + xm.z, nfk.z - x0.z, nhk.z - x0.z, x0.w - x0.z, w_t, w_s);
+                    a3 += term(xp.w - 2.f * x0.w + xm.w, nfk.w - x0.w, nhk.w - x0.w, nxk - x0.w, w_t, w_s);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(empty(slot));
+            if (++slot == S) { slot = 0; phase ^= 1; }
+        }
+        // ---- block sums by warp shuffles (bh, bw uniform: no divergence)
+        float p[4] = {a0, a1, a2, a3};
+        int nbt = 4;                                   // block partials per thread
+        if (g.bw >= 4) { p[0] = (a0 + a1) + (a2 + a3); nbt = 1; }
+        else if (g.bw == 2) { p[0] = a0 + a1; p[1] = a2 + a3; nbt = 2; }
+        for (int o = 8; o < 8 * g.bh; o <<= 1) {       // over the block's rows
+#pragma unroll
+            for (int j = 0; j < 4; ++j) p[j] += __shfl_xor_sync(0xFFFFFFFFu, p[j], o);
+        }
+        for (int o = 1; o < g.bw / 4; o <<= 1) p[0] += __shfl_xor_sync(0xFFFFFFFFu, p[0], o);
+        const bool writer = act && hr % g.bh == 0 && (g.bw <= 4 || ((lane & 7) & (g.bw / 4 - 1)) == 0);
+        if (writer) {
+            const int hb = h / g.bh;
+            const int rows = min(g.bh, g.H - hb * g.bh);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int ws = w + j * g.bw;
+                if (j >= nbt || ws >= g.W) break;
+                const int wb = ws / g.bw;
+                const int cols = min(g.bw, g.W - wb * g.bw);
+                const float cnt = (float)(K - 1) * (float)g.C * (float)(rows * cols);
+                scores[((size_t)f * g.nBh + hb) * g.nBw + wb] = p[j] / cnt;
+            }
+        }
+    }
+}
+
 int gcd(int a, int b) {
     while (b) { const int t = a % b; a = b; b = t; }
     return a;
@@ -359,16 +536,140 @@ bool plan(const jano_geom& gm, int K, int C, bool literal, AGeo& a) {
     return true;
 }
 
+// Frame-group plan.  Measured on B200 over the video latents of the pages'
+// configurations (units of 32 or 64 columns, 2 to 6 frames, rings of 2 or 3
+// stages): 32 columns, 3 frames and a 2-stage ring (15 KB stages, 64
+// registers a thread, so seven 128-thread CTAs fit an SM) is the fastest;
+// wider units or deeper rings leave fewer CTAs per SM and lose more than the
+// L2 bytes they save.  A latent with fewer than two such units per SM (the
+// image and tiny latents: one frame, or a few small frames) takes units of
+// one frame and a 4-stage ring instead, for more units in flight.  The unit
+// shape does not change a block's arithmetic (each thread adds its channels
+// and steps in the same order, and the shuffle tree is fixed), so every
+// shape, and every frame slab of a latent, gives the same bits.
+#ifndef JANO_ANALYZER_FG
+#define JANO_ANALYZER_FG 1
+#endif
+#ifndef JANO_ANALYZER_FG_WC
+#define JANO_ANALYZER_FG_WC 32
+#endif
+#ifndef JANO_ANALYZER_FG_G
+#define JANO_ANALYZER_FG_G 3
+#endif
+#ifndef JANO_ANALYZER_FG_S
+#define JANO_ANALYZER_FG_S 2
+#endif
+constexpr int kFgK = 5;
+static_assert(JANO_ANALYZER_FG_WC % 32 == 0 && JANO_ANALYZER_FG_WC + 4 <= 256, "unit width");
+static_assert(JANO_ANALYZER_FG_S >= 2 && JANO_ANALYZER_FG_S <= kMaxStages && kMaxStages >= 4, "ring depth");
+
+bool fg_eligible(const jano_geom& gm, int K, bool literal) {
+    if (!JANO_ANALYZER_FG || literal || K != kFgK || gm.bf != 1) return false;
+    if (gm.bh != 1 && gm.bh != 2 && gm.bh != 4) return false;
+    return gm.bw >= 1 && gm.bw <= 32 && (gm.bw & (gm.bw - 1)) == 0;
+}
+
+bool plan_fg(const jano_geom& gm, int K, int C, bool literal, int sms, FGeo& a) {
+    if (!fg_eligible(gm, K, literal)) return false;
+    a.C = C; a.F = gm.F; a.H = gm.H; a.W = gm.W;
+    a.bh = gm.bh; a.bw = gm.bw;
+    a.nBh = (gm.H + gm.bh - 1) / gm.bh;
+    a.nBw = (gm.W + gm.bw - 1) / gm.bw;
+    a.Wc = JANO_ANALYZER_FG_WC;
+    a.G = std::min(JANO_ANALYZER_FG_G, gm.F);
+    a.S = JANO_ANALYZER_FG_S;
+    a.LA = a.Wc + 4;
+    a.n_wc = (gm.W + a.Wc - 1) / a.Wc;
+    a.n_rg = (gm.H + 3) / 4;
+    long long n_units = (long long)((gm.F + a.G - 1) / a.G) * a.n_rg * a.n_wc;
+    if (n_units < 2ll * sms && a.G > 1) {
+        a.G = 1;
+        a.S = 4;
+        n_units = (long long)gm.F * a.n_rg * a.n_wc;
+    }
+    if (n_units > (1ll << 30)) return false;
+    a.n_units = (int)n_units;
+    a.n_warps = a.G * a.Wc / 32;
+    if ((a.n_warps + 1) * 32 > kFgMaxThreads) return false;
+    a.bytesA = a.LA * 5 * a.G * (K + 1) * 4;
+    a.bytesB = a.Wc * 4 * (K - 1) * 4;
+    a.offB = (a.bytesA + 127) / 128 * 128;
+    a.stage_bytes = (a.offB + a.bytesB + 127) / 128 * 128;
+    a.smem = a.S * a.stage_bytes + 16 * a.S + 16 + 128;
+    return a.smem <= 220 * 1024;
+}
+
 }  // namespace
 
 bool analyzer_supported(const jano_geom& g, int K, int C, bool literal) {
     AGeo a;
-    return plan(g, K, C, literal, a);
+    FGeo b;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return plan_fg(g, K, C, literal, sms, b) || plan(g, K, C, literal, a);
 }
+
+namespace {
+cudaError_t launch_fg(const float* lat, int K, int C, const jano_geom& gm, float w_t, float w_s,
+                      float* scores, int* err, cudaStream_t st, bool& taken) {
+    taken = false;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    FGeo a;
+    if (!plan_fg(gm, K, C, false, sms, a)) return cudaSuccess;
+    taken = true;
+    a.w_t = w_t;
+    a.w_s = w_s;
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorInvalidValue;
+    const cuuint64_t dims[5] = {(cuuint64_t)gm.W, (cuuint64_t)gm.H, (cuuint64_t)gm.F, (cuuint64_t)C,
+                                (cuuint64_t)(K + 1)};
+    const cuuint64_t strides[4] = {(cuuint64_t)gm.W * 4, (cuuint64_t)gm.H * gm.W * 4,
+                                   (cuuint64_t)gm.F * gm.H * gm.W * 4,
+                                   (cuuint64_t)C * gm.F * gm.H * gm.W * 4};
+    const cuuint32_t boxA[5] = {(cuuint32_t)a.LA, 5, (cuuint32_t)a.G, 1, (cuuint32_t)K + 1};
+    const cuuint32_t boxB[5] = {(cuuint32_t)a.Wc, 4, 1, 1, (cuuint32_t)(K - 1)};
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    CUtensorMap mA, mB;
+    if (fn(&mA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, const_cast<float*>(lat), dims, strides, boxA, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        fn(&mB, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, const_cast<float*>(lat), dims, strides, boxB, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    static DeviceOnce opted_in;
+    if (!opted_in.done(dev)) {
+        cudaError_t e = cudaFuncSetAttribute(analyzer_fg_kernel<kFgK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             224 * 1024);
+        if (e != cudaSuccess) return e;
+        opted_in.mark(dev);
+    }
+    const int threads = (a.n_warps + 1) * 32;
+    // resident CTAs per SM, asked once per device and unit shape
+    static std::atomic<int> occupancy[64][JANO_ANALYZER_FG_G + 1][kMaxStages + 1];   // by G and S
+    int per = dev < 64 ? occupancy[dev][a.G][a.S].load(std::memory_order_relaxed) : 0;
+    if (per < 1) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, analyzer_fg_kernel<kFgK>, threads,
+                                                          (size_t)a.smem) != cudaSuccess || per < 1)
+            per = 1;
+        if (dev < 64) occupancy[dev][a.G][a.S].store(per, std::memory_order_relaxed);
+    }
+    const int grid = a.n_units < per * sms ? a.n_units : per * sms;
+    analyzer_fg_kernel<kFgK><<<grid, threads, (size_t)a.smem, st>>>(mA, mB, a, scores, err);
+    return cudaGetLastError();
+}
+}  // namespace
 
 cudaError_t launch_block_scores(const float* lat, int K, int C, const jano_geom& gm,
                                 float w_t, float w_s, bool literal, float* scores, int* err,
                                 cudaStream_t st) {
+    if (!literal) {
+        bool taken = false;
+        const cudaError_t e = launch_fg(lat, K, C, gm, w_t, w_s, scores, err, st, taken);
+        if (taken) return e;
+    }
     AGeo a;
     if (!plan(gm, K, C, literal, a)) return cudaErrorInvalidValue;
     a.w_t = w_t;

@@ -78,11 +78,18 @@ def test_block_scores_match_oracle(J, name):
                                          ((3, 1, 2, 4, 20), (1, 4, 8)),     # bw = 8, partial
                                          ((4, 3, 3, 9, 520), (1, 4, 4)),    # wide rows: boxed chunks
                                          ((3, 2, 2, 6, 200), (2, 4, 8)),    # whole rows, bf = 2
-                                         # K = 5 with 1x4x4 blocks (the frame-run path):
+                                         # K = 5, blocks of one frame (the frame-group form):
                                          ((6, 2, 1, 9, 20), (1, 4, 4)),     # F = 1, partial row, odd blocks
-                                         ((6, 3, 5, 14, 200), (1, 4, 4)),   # two column chunks, ragged
-                                         ((6, 2, 11, 8, 328), (1, 4, 4)),   # runs of several frames
-                                         ((6, 1, 21, 6, 48), (1, 4, 4))])   # many runs, short rows
+                                         ((6, 3, 5, 14, 200), (1, 4, 4)),   # several column chunks, ragged
+                                         ((6, 2, 11, 8, 328), (1, 4, 4)),   # frame groups, wide rows
+                                         ((6, 1, 21, 6, 48), (1, 4, 4)),    # many frame groups, short rows
+                                         ((6, 2, 7, 13, 52), (1, 4, 4)),    # ragged H, W and last frame group
+                                         ((6, 3, 5, 10, 96), (1, 2, 8)),    # bh = 2, bw = 8
+                                         ((6, 2, 4, 9, 40), (1, 1, 1)),     # one-element blocks
+                                         ((6, 2, 3, 7, 200), (1, 4, 32)),   # bw = 32, ragged last block
+                                         ((6, 2, 9, 6, 36), (1, 2, 16)),    # bw = 16, ragged last block
+                                         ((6, 2, 2, 5, 4), (1, 4, 4)),      # one float4 per row
+                                         ((6, 2, 3, 11, 24), (1, 2, 2))])   # 2x2 blocks, ragged rows
 def test_block_scores_edge_geometries(J, shape, block):
     g = np.random.default_rng(sum(shape))
     lat = g.standard_normal(shape).astype(np.float32)
