@@ -10,14 +10,20 @@
 // so no step has to wait on another and no tile on another:
 //   1. count   one CTA per 1024-token tile: token level (from the block map)
 //              stored to scratch, per-level counts of the tile via warp ballots;
-//   2. write   one CTA per tile: its per-level prefix over the earlier tiles
-//              and the level totals by a block reduction over the tile counts,
-//              the step offsets in closed form from those totals, the tile's
-//              tokens ranked once in each of the four possible due sets
-//              (ballot + popc + one warp scan per set), then ascending stores
-//              of the due ids of every step.
+//   2. write   one CTA per (tile, chunk of steps): its per-level prefix over
+//              the earlier tiles and the level totals by a block reduction
+//              over the tile counts, the step offsets in closed form from
+//              those totals, the tile's tokens ranked once in each of the four
+//              possible due sets (ballot + popc + one warp scan per set), then
+//              ascending stores of the due ids of the chunk's steps.  The
+//              chunks spread the stores of the 50 steps over every SM.  It is
+//              launched as a programmatic dependent of the count pass: its
+//              CTAs become resident while the count pass runs and wait
+//              (griddepcontrol.wait) for its results before reading them.
 // Scratch (caller-provided): token levels [n_tokens] u8 and tile counts
 // [3][n_tiles] int32, each part 16-byte aligned.
+#include <algorithm>
+
 #include "jano_common.cuh"
 
 namespace jano {
@@ -63,6 +69,9 @@ __device__ __forceinline__ void step_due(int s, const jano_sched_cfg& c, bool& d
 __global__ void __launch_bounds__(kTile)
 count_kernel(const uint8_t* __restrict__ block_levels, Geo g, int n_tokens,
              uint8_t* __restrict__ token_levels, Ws ws, int n_tiles, int* err) {
+    // the write pass may be scheduled now; it reads nothing of ours before
+    // this grid has completed (griddepcontrol.wait)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ int wc[3][32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t = blockIdx.x * kTile + tid;
@@ -132,6 +141,11 @@ write_kernel(Ws ws, int n_tokens, int n_tiles, jano_sched_cfg c,
     __shared__ unsigned char s_set[kStepChunk];  // their due sets
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tile = blockIdx.x;
+    // this CTA's steps: chunk blockIdx.y of gridDim.y
+    const int s_lo = (int)((long long)c.T * blockIdx.y / gridDim.y);
+    const int s_hi = (int)((long long)c.T * (blockIdx.y + 1) / gridDim.y);
+    // the count pass's token levels and tile counts are complete and visible after this
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // ---- per-level prefix over earlier tiles and totals over all tiles
     int pre[3] = {0, 0, 0}, tot[3] = {0, 0, 0};
@@ -194,11 +208,11 @@ write_kernel(Ws ws, int n_tokens, int n_tiles, jano_sched_cfg c,
     for (int set = 0; set < 4; ++set)
         pos[set] = s_pre[2] + ((set & 1) ? s_pre[1] : 0) + ((set & 2) ? s_pre[0] : 0) +
                    wpre[set][warp] + rank[set];
-    if (tile == 0 && tid == 0) offsets[0] = 0;
+    if (tile == 0 && s_lo == 0 && tid == 0) offsets[0] = 0;
 
-    // ---- every step's part of this tile, steps staged in chunks
-    for (int s0 = 0; s0 < c.T; s0 += kStepChunk) {
-        const int ns = min(kStepChunk, c.T - s0);
+    // ---- this tile's part of the chunk's steps, staged kStepChunk at a time
+    for (int s0 = s_lo; s0 < s_hi; s0 += kStepChunk) {
+        const int ns = min(kStepChunk, s_hi - s0);
         __syncthreads();                     // the previous chunk's entries are consumed
         if (tid < ns) {
             const int s = s0 + tid;
@@ -247,8 +261,24 @@ cudaError_t launch_build_schedule(const uint8_t* block_levels, const jano_geom& 
     const Ws ws = carve(ws_base, n_tokens, n_tiles);
     count_kernel<<<n_tiles, kTile, 0, st>>>(block_levels, geo, n_tokens, token_levels, ws,
                                              n_tiles, err);
-    write_kernel<<<n_tiles, kTile, 0, st>>>(ws, n_tokens, n_tiles, c, offsets, idx);
-    return cudaGetLastError();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // step chunks: enough (tile, chunk) CTAs for two per SM, at most one chunk per step
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int chunks = std::max(1, std::min(c.T, (2 * sms + n_tiles - 1) / n_tiles));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)n_tiles, (unsigned)chunks, 1);
+    cfg.blockDim = dim3(kTile, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, write_kernel, ws, n_tokens, n_tiles, c, offsets, idx);
 }
 
 }  // namespace jano

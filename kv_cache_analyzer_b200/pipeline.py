@@ -94,7 +94,9 @@ class HotPath:
     def plan(self):
         """Run a1..a3 once and read the CSR offsets back (one D2H per generation)."""
         self.run_plan_kernels()
-        self.host_offsets = self.offsets.to("cpu", non_blocking=False).tolist()
+        # the copy is ordered after the kernels on their own stream
+        with torch.cuda.stream(self.stream):
+            self.host_offsets = self.offsets.to("cpu", non_blocking=False).tolist()
         return self.host_offsets
 
     def due(self, step: int):

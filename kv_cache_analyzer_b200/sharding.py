@@ -167,7 +167,9 @@ class ShardedHotPath:
 
     def plan(self):
         self.run_plan_kernels()
-        self.host_offsets = self.offsets.to("cpu", non_blocking=False).tolist()
+        # the copy is ordered after the kernels on their own stream
+        with torch.cuda.stream(self.stream):
+            self.host_offsets = self.offsets.to("cpu", non_blocking=False).tolist()
         return self.host_offsets
 
     def due(self, step: int):
