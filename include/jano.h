@@ -138,8 +138,8 @@ JANO_API jano_status jano_block_scores_literal(const float *lat, int K, int C, c
  * scores  device fp32 [n_blocks] (any finite values).
  * levels  device uint8 [n_blocks], written with 1, 2 or 3.
  * A NaN or infinite score raises JANO_ENONFINITE on the device error word
- * and leaves `levels` unspecified.  One cluster of 8 thread blocks; no
- * scratch memory.
+ * and leaves `levels` unspecified.  One thread-block cluster (16 blocks
+ * where the device runs clusters of that size, else 8); no scratch memory.
  * ---------------------------------------------------------------------- */
 JANO_API jano_status jano_classify(const float *scores, int n_blocks, float frac_active,
                           float frac_static, uint8_t *levels, void *stream);

@@ -142,6 +142,32 @@ def test_classify_ties_and_sizes(J, n):
         np.testing.assert_array_equal(got, oracle.classify(s, fa, fs), err_msg=f"{fa},{fs}")
 
 
+@pytest.mark.parametrize("dist", ["normal", "outliers", "lognormal", "denormal", "narrow", "mixed_sign_zero"])
+def test_classify_value_domain_first_pass(J, dist):
+    # the first pass bins float values: few candidates (direct rank), crowded
+    # bins (radix over the gathered candidates) and bins beyond the gather
+    # buffers (the select starts over on the order keys), all against the oracle
+    g = np.random.default_rng(len(dist))
+    n = 75_600
+    if dist == "normal":
+        s = g.standard_normal(n)
+    elif dist == "outliers":                        # a few huge values: one bin holds almost all
+        s = g.standard_normal(n)
+        s[g.choice(n, 5, replace=False)] = [1e30, -1e30, 3e29, 1e25, -7e28]
+    elif dist == "lognormal":
+        s = g.lognormal(0.0, 4.0, n)
+    elif dist == "denormal":                        # subnormal floats only
+        s = g.integers(1, 1 << 20, n).astype(np.uint32).view(np.float32).astype(np.float64)
+    elif dist == "narrow":                          # a handful of distinct floats near 1
+        s = 1.0 + g.integers(0, 40, n) * 2.0 ** -23
+    else:                                           # signed zeros and small integers
+        s = g.choice([-0.0, 0.0, -1.0, 1.0, 2.0], n) + g.choice([0.0, 0.25], n)
+    s = s.astype(np.float32)
+    for fa, fs in [(0.25, 0.45), (0.3, 0.4), (0.0, 0.5), (0.5, 0.0), (0.01, 0.98)]:
+        got = J.classify(torch.from_numpy(s).cuda(), fa, fs).cpu().numpy()
+        np.testing.assert_array_equal(got, oracle.classify(s, fa, fs), err_msg=f"{dist} {fa},{fs}")
+
+
 def test_classify_all_equal_split_by_index(J):
     got = J.classify(torch.zeros(10, device="cuda"), 0.3, 0.3).cpu().numpy()
     np.testing.assert_array_equal(got, [1, 1, 1, 2, 2, 2, 2, 3, 3, 3])
