@@ -557,6 +557,12 @@ def run_gpu(args, w, rank, world, local_rank, dist):
                "h2d_bytes_per_step": HotPath.h2d_bytes(host),
                "d2h_bytes_per_step": host_out.numel() * host_out.element_size()}
 
+    # ---- the same step replayed from a CUDA graph, and the launch-bound plan
+    # kernels timed in graphs of back-to-back launches (every rank alike)
+    graph = None
+    if not args.no_graph:
+        graph = measure_graphs(J, hp, step, stream, args.steps, flops, world, dist, dev)
+
     if rank != 0:
         return 0
 
@@ -578,6 +584,9 @@ def run_gpu(args, w, rank, world, local_rank, dist):
     }
     for k in ("block_scores", "kv_scatter"):
         kernels[k]["frac_of_hbm"] = kernels[k]["GB/s"] / hbm
+    if graph is not None:
+        kernels["classify"]["graph_us"] = graph.pop("classify_us")
+        kernels["build_schedule"]["graph_us"] = graph.pop("build_schedule_us")
     kernels["active_attention"]["frac_of_burst_peak"] = att_tflops / pk["bf16_tflops"]
     roofline = {"bound": "tensor", "achieved": att_tflops, "peak": bf16_sus, "unit": "TFLOP/s",
                 "frac": att_tflops / bf16_sus,
@@ -608,7 +617,7 @@ def run_gpu(args, w, rank, world, local_rank, dist):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": cfg, "roofline": roofline, "cpu_baseline": cpu,
             "e2e": e2e, "gpu_launches": (KERNELS_PER_STEP + (1 if hp.last_split > 1 else 0)) * args.steps, "clocks": clk.summary(),
-            "kernels": kernels, "next_rows": next_rows,
+            "kernels": kernels, "graph": graph, "next_rows": next_rows,
             "peaks": {"source": pk_src, "hbm_gbs": hbm,
                                           "bf16_tflops": pk["bf16_tflops"],
                                           "bf16_tflops_sustained": bf16_sus}}
@@ -617,6 +626,46 @@ def run_gpu(args, w, rank, world, local_rank, dist):
 
 
 # ------------------------------------------------------------------ other measurements
+def measure_graphs(J, hp, step, stream, steps, flops, world, dist, dev, repeat=20, reps=5):
+    """The step captured once as a CUDA graph and replayed `steps` times (no
+    host launches; device time by events on the stream, max over ranks), and
+    classify and the schedule each captured as `repeat` back-to-back
+    launches (per launch: replay time / repeat; their inputs are a few
+    hundred KB, resident in L2 after the first launch, as in the step)."""
+    import torch
+    g = hp.capture_step(step)
+    cls = hp.capture_repeated(
+        lambda s: J.jano_classify(hp.field, hp.field.numel(), hp.frac_active, hp.frac_static, hp.levels, s),
+        repeat)
+    sch = hp.capture_repeated(
+        lambda s: J.jano_build_schedule(hp.levels, hp._tgc, hp._sc, hp.offsets, hp.idx, hp.idx.numel(),
+                                        hp.token_levels, hp.ws, hp.ws_bytes, s),
+        repeat)
+
+    def replay_ms(graph, n):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                graph.replay()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(n):
+                graph.replay()
+            b.record(stream)
+        stream.synchronize()
+        return a.elapsed_time(b)
+
+    step_ms = max_over_ranks(replay_ms(g, steps), dist, dev) / steps
+    cls_us = replay_ms(cls, reps) / (reps * repeat) * 1e3
+    sch_us = replay_ms(sch, reps) / (reps * repeat) * 1e3
+    _raise_device_error(J, stream, "graph replays")
+    del g, cls, sch
+    return {"step_ms": step_ms, "TFLOP/s": whole_job_tflops(flops, world, step_ms), "replays": steps,
+            "classify_us": cls_us, "build_schedule_us": sch_us, "launches_per_graph": repeat,
+            "note": "the timed step replayed from one CUDA graph; classify and schedule per launch "
+                    "inside graphs of back-to-back launches (no host work between launches)"}
+
+
+
 def _events_ms(fn, stream, reps, warm=2, pick="median"):
     """Device time of fn() on `stream` by CUDA events (after `warm` calls)."""
     import torch
@@ -926,6 +975,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=0,
                     help="attention rows per oracle sample (0: 8 for the GPU arm's baseline, "
                          "sized from --steps/--warmup for --impl reference)")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replays of the step")
     ap.add_argument("--no-next", action="store_true",
                     help="skip the projections measured beside the step")
     ap.add_argument("--mode", default="step",

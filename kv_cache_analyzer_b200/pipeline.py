@@ -25,7 +25,7 @@ from . import (Geometry, Schedule, SplitWorkspace, attention_auto, jano_block_sc
                jano_build_schedule, jano_build_schedule_workspace_bytes,
                jano_classify, jano_kv_scatter)
 
-KERNELS_PER_STEP = 7      # scores 1 + classify 1 + schedule 3 + scatter 1 + attention 1
+KERNELS_PER_STEP = 6      # scores 1 + classify 1 + schedule 2 + scatter 1 + attention 1
                           # (attention 2 when its keys are split: + the merge pass)
 
 
@@ -118,6 +118,31 @@ class HotPath:
                                          self.heads, self.d, self.out, s, self.att_ws)
         if ev[5] is not None: ev[5].record(s)
         return n_act
+
+    def capture_step(self, step: int) -> torch.cuda.CUDAGraph:
+        """a1..a5 of sampling step `step` captured once as a CUDA graph on the
+        hot path's stream (which must not be the default stream); replay()
+        re-runs the step with no host launches.  One ordinary pass runs first,
+        so that everything the entry points make lazily (the device error
+        word, shared-memory opt-ins, the key-split workspace) exists before
+        the capture."""
+        self.run_step_kernels(step)
+        self.stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            self.run_step_kernels(step)
+        return g
+
+    def capture_repeated(self, fn, times: int) -> torch.cuda.CUDAGraph:
+        """`times` back-to-back calls of fn(stream) captured as one graph (the
+        launch-bound plan kernels timed without per-launch host work)."""
+        fn(self.stream)
+        self.stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            for _ in range(times):
+                fn(self.stream)
+        return g
 
     def step_from_host(self, step: int, host: dict, host_out: torch.Tensor):
         """The same pass with this step's inputs copied in from host memory
