@@ -973,8 +973,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=0,
-                    help="attention rows per oracle sample (0: 8 for the GPU arm's baseline, "
-                         "sized from --steps/--warmup for --impl reference)")
+                    help="attention rows per oracle sample of --impl reference (0: sized from "
+                         "--steps/--warmup so the run ends within minutes)")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replays of the step")
     ap.add_argument("--no-next", action="store_true",
                     help="skip the projections measured beside the step")
